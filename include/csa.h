@@ -1,0 +1,257 @@
+/*
+ * csa.h -- C ABI of libcsa: the CSA / HCA attention hot path on B200 (sm_100a).
+ *
+ * The operation.  The DeepSeek-V4 summary page (b-lab.team), section "Core
+ * Methodological Innovations", item 1 "Hybrid Attention Architecture (CSA
+ * and HCA)", states the method this library computes:
+ *   - CSA bullet: the KV cache is compressed by a factor m by combining
+ *     adjacent entries; a "Lightning Indexer" computes scores from low-rank
+ *     projections of the query hidden state h_t and selects the top-k most
+ *     relevant compressed KV blocks, which are then attended (sparse
+ *     attention).
+ *   - HCA bullet: a stronger compression by m' >> m, with dense attention
+ *     over all remaining entries; both mechanisms add a sliding window of
+ *     local (uncompressed) KV entries.
+ * Where the page is silent this library takes the readings below, and every
+ * call states the one it uses:
+ *   R1 pooling: C[j][c] = sum_{i<m} a[i][c] X[j m + i][c], with a[.][c] the
+ *      softmax over the m positions of per-position, per-channel logits z.
+ *   R2 a trailing partial block (< m rows) is not compressed.
+ *   R3 indexer: u = W_dq h (rank r), q_h = W_uq[h] u (64-d per head),
+ *      w = W_w h, score S_j = sum_h w_h max(0, q_h . k_j) (times the row
+ *      scale s_j for FP8 keys); no extra scale, no softmax.
+ *   R4 causality: block j (raw tokens [j m, j m + m)) is visible to a query
+ *      at position p iff j < (p + 1) / m; the window is the raw rows s with
+ *      p - W < s <= p, s >= 0.
+ *   R5 top-k order: score descending, then block index ascending; fewer
+ *      than k visible blocks pad the row with -1.
+ *   R6 attention: K = V = the 128-d latent row, logits scale * q_h . x,
+ *      softmax over {selected compressed rows} + {window rows} (a block
+ *      inside the window is attended in both forms).
+ *
+ * Conventions (all calls):
+ *   - Every data pointer is a DEVICE pointer owned by the caller (lengths and
+ *     sizes are host ints).  The library allocates nothing and keeps no
+ *     per-call state; scratch lives in the caller's workspace.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *     and returns a csa_status.  Argument errors are detected before any
+ *     launch and have no side effects; csa_last_error() gives the detail.
+ *   - bf16 = IEEE-754 binary16 with 8 exponent bits (bfloat16) stored as
+ *     2-byte words; E4M3 = OCP OFP8 E4M3 (max 448) stored as bytes.
+ *   - Arrays are row-major and each row is contiguous; per-sequence strides
+ *     are given in ELEMENTS.  Rows must be 16-byte aligned (base pointers
+ *     16-byte aligned, strides multiples of 8 bf16 / 16 bytes).
+ *   - A query t belongs to sequence q_seq[t] and sits at absolute position
+ *     q_pos[t] (device int32 arrays).  At decode q_pos[t] = length - 1 and
+ *     the token's own raw row is already in the raw cache.
+ *   - Results are deterministic and batch-invariant: a query's outputs are
+ *     bitwise the same whatever other queries share the call, and across
+ *     runs (fixed split sizes, no floating-point atomics).
+ *   - Device-side anomalies (an out-of-range block index) never trap: the
+ *     offending entry is skipped and a bit is set in a status word at the
+ *     start of the workspace; csa_status_check() reads and clears it.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t (CUDA defines it as struct CUstream_st*). */
+struct CUstream_st;
+typedef struct CUstream_st* csa_stream_t;
+
+typedef enum csa_status {
+    CSA_OK = 0,
+    CSA_ERR_NULL = 1,         /* a required pointer is NULL */
+    CSA_ERR_SHAPE = 2,        /* inconsistent or negative sizes / strides */
+    CSA_ERR_UNSUPPORTED = 3,  /* size outside the supported ranges below */
+    CSA_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than required */
+    CSA_ERR_CUDA = 5,         /* a CUDA launch or runtime call failed */
+    CSA_ERR_TIMEOUT = 6,      /* a bounded device wait gave up */
+    CSA_ERR_DEVICE = 7,       /* device status word had anomaly bits set */
+    CSA_ERR_ALIGN = 8         /* a pointer or stride breaks 16-byte alignment */
+} csa_status;
+
+enum { CSA_FMT_BF16 = 0, CSA_FMT_FP8E4M3 = 1 };
+
+/* Device status bits (see csa_status_check). */
+enum { CSA_DEV_BAD_INDEX = 1u, CSA_DEV_TIMEOUT = 2u };
+
+/* Supported ranges (anything else returns CSA_ERR_UNSUPPORTED). */
+#define CSA_D_LATENT 128   /* latent KV row width (bf16) */
+#define CSA_D_INDEX 64     /* indexer key / query head width */
+#define CSA_MAX_M 256      /* compression factor m: 1..256 */
+#define CSA_MAX_HI 16      /* indexer heads: 1..16 */
+#define CSA_MAX_K 2048     /* top-k: 1..2048 */
+#define CSA_MAX_W 1024     /* window: 0..1024 */
+/* attention heads H: 16, 32, 48, ..., 128 (a multiple of 16) */
+
+/* Human-readable name of a status code (static string). */
+const char* csa_status_string(csa_status s);
+
+/* Detail of the last error on the calling host thread (static per thread;
+ * empty string after a successful call). */
+const char* csa_last_error(void);
+
+/* Number of kernels this library has launched since it was loaded (all
+ * threads).  Used to count device launches in a timed region. */
+uint64_t csa_launch_count(void);
+
+/* Bytes reserved at the start of every workspace for the status word. */
+#define CSA_WS_HEADER_BYTES 256
+
+/* Zero the status word of a freshly allocated workspace (async). */
+csa_status csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* Synchronise `stream`, read the workspace's status word, clear it.
+ * Returns CSA_OK, or CSA_ERR_DEVICE with the bits in csa_last_error(). */
+csa_status csa_status_check(void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* 1. Compression (CSA bullet: "combining adjacent entries"; HCA bullet:  */
+/*    the same with m' >> m).  Readings R1, R2.                          */
+/* ------------------------------------------------------------------ */
+/*
+ * raw        bf16 [B][raw_seq_stride/d][d], row s of sequence b at
+ *            raw + b*raw_seq_stride + s*d.
+ * lens       device int32 [B]: raw rows present per sequence.
+ * d          128 (latent KV) or 64 (indexer keys).
+ * m          1..256.
+ * pool_logits device fp32 [m][d]: z; the weights are softmax over i of z[i][c]
+ *            (computed in fp32 inside the call; -inf logits give exact zeros).
+ * blk_lo, blk_hi
+ *            blk_lo >= 0: compress blocks j in [blk_lo, min(blk_hi, lens[b]/m)).
+ *            blk_lo == -1: compress the last blk_hi complete blocks of each
+ *            sequence (decode: blk_hi = 1 refreshes the newest block).
+ * out        bf16 [B][.][d] (out_fmt CSA_FMT_BF16) or E4M3 bytes (CSA_FMT_FP8E4M3,
+ *            d = 64 only), row j at out + b*out_seq_stride + j*d.
+ * out_scale  fp32 [B][scale_seq_stride] for E4M3 (NULL for bf16): s_j = amax_j/448
+ *            of the bf16-rounded row (1 if the row is all zeros), codes =
+ *            e4m3_rn_satfinite(x / s_j) in fp32.
+ * Accumulation: fp32, one FMA per position in order i = 0..m-1; bf16 output
+ * rounded to nearest even.  Blocks outside the range are not written.
+ */
+csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* lens,
+                        int B, int d, int m, const float* pool_logits,
+                        int blk_lo, int blk_hi,
+                        void* out, int64_t out_seq_stride, int out_fmt,
+                        float* out_scale, int64_t scale_seq_stride,
+                        csa_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* 2. Lightning indexer (CSA bullet: scores from low-rank projections of  */
+/*    h_t, top-k most relevant compressed blocks).  Readings R3-R5.       */
+/* ------------------------------------------------------------------ */
+
+/* Workspace for csa_index_query / csa_index_select / csa_index_topk. */
+size_t csa_index_workspace_size(int T, int r, int Hi, int k, int max_blocks);
+
+/*
+ * Indexer query projection.  h bf16 [T][D]; W_dq bf16 [r][D]; W_uq bf16
+ * [Hi*64][r]; W_w bf16 [Hi][D].  Outputs q fp32 [T][Hi][64] and w fp32 [T][Hi]
+ * (not rounded further).  u = W_dq h is kept in fp32 (workspace).
+ * Constraints: D % 8 == 0, r % 8 == 0, 1 <= Hi <= 16.
+ */
+csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
+                           const void* W_dq, const void* W_uq, const void* W_w,
+                           float* q_out, float* w_out,
+                           void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/*
+ * Full indexer score matrix (for inspection and parity checks): scores fp32
+ * [T][max_blocks], S[t][j] for j < min(V(t), max_blocks), NaN elsewhere.
+ * kidx: bf16 [B][.][64] (CSA_FMT_BF16) or E4M3 [B][.][64] with kidx_scale
+ * fp32 [B][scale_seq_stride] (CSA_FMT_FP8E4M3).  Uses the same scoring
+ * arithmetic as csa_index_select.
+ */
+csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq,
+                            const int32_t* q_pos, int T, int Hi,
+                            const void* kidx, int kidx_fmt, const float* kidx_scale,
+                            int64_t kidx_seq_stride, int64_t scale_seq_stride,
+                            int m, int max_blocks, float* scores, csa_stream_t stream);
+
+/*
+ * Score every visible block and select the per-query top-k (R5): out_idx
+ * int32 [T][k] sorted by (score desc, index asc), padded with -1;
+ * out_score fp32 [T][k] (NaN at padding) or NULL.  max_blocks bounds V(t)
+ * for every query (blocks past it are ignored).  The scores are never
+ * materialised: each CTA keeps its chunk's scores on chip and emits its
+ * exact local top-k, which later stages merge.  Equivalent to
+ * csa_index_stage_score followed by csa_index_stage_merge.
+ */
+csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq,
+                            const int32_t* q_pos, int T, int Hi,
+                            const void* kidx, int kidx_fmt, const float* kidx_scale,
+                            int64_t kidx_seq_stride, int64_t scale_seq_stride,
+                            int m, int max_blocks, int k,
+                            int32_t* out_idx, float* out_score,
+                            void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* First stage of csa_index_select: the streaming score kernel, writing the
+ * per-chunk exact top-k candidates into the workspace. */
+csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* q_seq,
+                                 const int32_t* q_pos, int T, int Hi,
+                                 const void* kidx, int kidx_fmt, const float* kidx_scale,
+                                 int64_t kidx_seq_stride, int64_t scale_seq_stride,
+                                 int m, int max_blocks, int k,
+                                 void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* Second stage: merge the candidates left in the workspace by
+ * csa_index_stage_score (same T, max_blocks, k) into out_idx / out_score. */
+csa_status csa_index_stage_merge(int T, int max_blocks, int k,
+                                 int32_t* out_idx, float* out_score,
+                                 void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* csa_index_query followed by csa_index_select. */
+csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq,
+                          const void* W_uq, const void* W_w,
+                          const int32_t* q_seq, const int32_t* q_pos, int T, int Hi,
+                          const void* kidx, int kidx_fmt, const float* kidx_scale,
+                          int64_t kidx_seq_stride, int64_t scale_seq_stride,
+                          int m, int max_blocks, int k,
+                          int32_t* out_idx, float* out_score,
+                          void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------ */
+/* 3. Attention (CSA: sparse over the selected blocks + window; HCA:      */
+/*    dense over all visible compressed rows + window).  Reading R6.      */
+/* ------------------------------------------------------------------ */
+
+/* Workspace for csa_sparse_attend (max_rows = k + W) and hca_attend
+ * (max_rows = max_blocks + W). */
+size_t csa_attend_workspace_size(int T, int H, int max_rows);
+
+/*
+ * q bf16 [T][H][128]; comp bf16 compressed latent rows [B][.][128] (row j at
+ * comp + b*comp_seq_stride + j*128); raw bf16 raw latent rows, same layout;
+ * idx int32 [T][k] block indices (entries < 0 are skipped; entries >= V(t)
+ * are skipped and flagged CSA_DEV_BAD_INDEX).  out bf16 [T][H][128];
+ * lse fp32 [T][H] (natural log of the softmax denominator, -inf for an
+ * empty set) or NULL.  An empty attended set gives out = 0.
+ * fp32 logits, softmax and accumulation; split-K over fixed 128-row
+ * splits merged in a fixed order.
+ */
+csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
+                             int T, int H, const void* comp, int64_t comp_seq_stride,
+                             const void* raw, int64_t raw_seq_stride, int m,
+                             const int32_t* idx, int k, int W, float scale,
+                             void* out, float* lse,
+                             void* ws, size_t ws_bytes, csa_stream_t stream);
+
+/* HCA: as csa_sparse_attend with the attended compressed rows being every
+ * visible block j < min(V(t), max_blocks) (m = m'). */
+csa_status hca_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
+                      int T, int H, const void* comp, int64_t comp_seq_stride,
+                      const void* raw, int64_t raw_seq_stride, int m, int max_blocks,
+                      int W, float scale, void* out, float* lse,
+                      void* ws, size_t ws_bytes, csa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

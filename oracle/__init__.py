@@ -1,0 +1,208 @@
+"""CPU oracle for the CSA / HCA hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the bench's CPU-baseline /
+reference leg may import this package.  The product path (the CUDA library
+and its binding in ``long_context_sparse_03_b200``) never touches it, and
+the two share no code.
+
+The oracle is plain C (``oracle.c``) in double precision; this module only
+builds it with gcc and marshals numpy arrays through ctypes.  Each function
+states what it computes; the C file cites the passage it follows (the
+DeepSeek-V4 summary page, "Core Methodological Innovations", item 1, the CSA
+and HCA bullets) and the readings taken where the pages are silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_BUILD = _HERE / "_build"
+
+FMT_BF16 = 0
+FMT_FP8E4M3 = 1
+
+
+def build(plant: int = 0, force: bool = False) -> Path:
+    """Compile oracle.c into a shared library (``plant`` > 0 plants a
+    deliberate mistake, for the tests that show the pins catch it)."""
+    _BUILD.mkdir(exist_ok=True)
+    name = "liboracle.so" if plant == 0 else f"liboracle_plant{plant}.so"
+    out = _BUILD / name
+    src = _HERE / "oracle.c"
+    if force or not out.exists() or out.stat().st_mtime < max(
+            src.stat().st_mtime, (_HERE / "oracle.h").stat().st_mtime):
+        tmp = out.with_suffix(f".{os.getpid()}.tmp")
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+               "-fno-fast-math", "-ffp-contract=off", f"-DORACLE_PLANT={plant}",
+               "-o", str(tmp), str(src), "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, out)
+    return out
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_L = ctypes.c_int64
+_D = ctypes.c_double
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """ctypes handle on one build of the oracle library."""
+
+    def __init__(self, plant: int = 0):
+        self.lib = ctypes.CDLL(str(build(plant)))
+        L = self.lib
+        L.oracle_double_to_bf16.restype = ctypes.c_uint16
+        L.oracle_double_to_bf16.argtypes = [_D]
+        L.oracle_bf16_to_double.restype = _D
+        L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.oracle_e4m3_to_double.restype = _D
+        L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_float_to_e4m3_satfinite.restype = ctypes.c_uint8
+        L.oracle_float_to_e4m3_satfinite.argtypes = [ctypes.c_float]
+        L.oracle_pool_weights.argtypes = [_P, _I, _I, _P]
+        L.oracle_compress.argtypes = [_P, _L, _P, _I, _I, _I, _P, _I, _I, _I, _P, _L, _P, _L]
+        L.oracle_index_query.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P]
+        L.oracle_index_scores.argtypes = [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _P]
+        L.oracle_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
+        L.oracle_sparse_attend.argtypes = [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _P, _I, _I, _D, _P, _P]
+        L.oracle_hca_attend.argtypes = [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _I, _D, _P, _P]
+        L.oracle_num_threads.restype = _I
+
+    # -- number formats ------------------------------------------------
+    def to_bf16(self, x: np.ndarray) -> np.ndarray:
+        """Round float64 values to bf16 bit patterns (uint16), RNE."""
+        x = np.asarray(x, dtype=np.float64)
+        f = np.vectorize(self.lib.oracle_double_to_bf16, otypes=[np.uint16])
+        return f(x) if x.size else x.astype(np.uint16)
+
+    def e4m3_encode(self, v: np.ndarray) -> np.ndarray:
+        v = np.asarray(v, dtype=np.float32)
+        f = np.vectorize(lambda a: self.lib.oracle_float_to_e4m3_satfinite(float(a)), otypes=[np.uint8])
+        return f(v)
+
+    def e4m3_decode(self, c: np.ndarray) -> np.ndarray:
+        c = np.asarray(c, dtype=np.uint8)
+        f = np.vectorize(lambda a: self.lib.oracle_e4m3_to_double(int(a)), otypes=[np.float64])
+        return f(c)
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    # -- the method ----------------------------------------------------
+    def pool_weights(self, z: np.ndarray) -> np.ndarray:
+        z = np.ascontiguousarray(z, dtype=np.float32)
+        m, d = z.shape
+        a = np.empty((m, d), np.float64)
+        self.lib.oracle_pool_weights(_ptr(z), m, d, _ptr(a))
+        return a
+
+    def compress(self, raw: np.ndarray, lens: np.ndarray, z: np.ndarray, blk_lo: int,
+                 blk_hi: int, out_fmt: int = FMT_BF16, out=None, out_scale=None):
+        """raw: uint16 [B][Lmax][d] bf16 bits; z: float32 [m][d].
+        Returns (out, scale): out uint16 [B][Nmax][d] (bf16) or uint8 (E4M3)."""
+        raw = np.ascontiguousarray(raw, dtype=np.uint16)
+        B, Lmax, d = raw.shape
+        z = np.ascontiguousarray(z, dtype=np.float32)
+        m = z.shape[0]
+        lens = np.ascontiguousarray(lens, dtype=np.int32)
+        nmax = max(1, Lmax // m)
+        if out is None:
+            out = np.zeros((B, nmax, d), np.uint16 if out_fmt == FMT_BF16 else np.uint8)
+        if out_fmt == FMT_FP8E4M3 and out_scale is None:
+            out_scale = np.zeros((B, out.shape[1]), np.float32)
+        self.lib.oracle_compress(_ptr(raw), Lmax * d, _ptr(lens), B, d, m, _ptr(z), blk_lo, blk_hi,
+                                 out_fmt, _ptr(out), out.shape[1] * d, _ptr(out_scale),
+                                 0 if out_scale is None else out_scale.shape[1])
+        return out, out_scale
+
+    def index_query(self, h, W_dq, W_uq, W_w):
+        """h uint16 [T][D]; W_dq [r][D]; W_uq [Hi*64][r]; W_w [Hi][D] (bf16 bits).
+        Returns q float64 [T][Hi][64], w float64 [T][Hi]."""
+        h = np.ascontiguousarray(h, dtype=np.uint16)
+        T, D = h.shape
+        r = W_dq.shape[0]
+        Hi = W_w.shape[0]
+        q = np.empty((T, Hi, 64), np.float64)
+        w = np.empty((T, Hi), np.float64)
+        args = [np.ascontiguousarray(x, dtype=np.uint16) for x in (W_dq, W_uq, W_w)]
+        self.lib.oracle_index_query(_ptr(h), T, D, r, Hi, *[_ptr(x) for x in args], _ptr(q), _ptr(w))
+        return q, w
+
+    def index_scores(self, q, w, q_seq, q_pos, kidx, m, max_blocks, kidx_fmt=FMT_BF16,
+                     kidx_scale=None):
+        """kidx: uint16 (bf16) or uint8 (E4M3) [B][N][64]; returns float64 [T][max_blocks]
+        (NaN for invisible blocks)."""
+        q = np.ascontiguousarray(q, dtype=np.float64)
+        w = np.ascontiguousarray(w, dtype=np.float64)
+        T, Hi, _ = q.shape
+        kidx = np.ascontiguousarray(kidx)
+        q_seq = np.ascontiguousarray(q_seq, dtype=np.int32)
+        q_pos = np.ascontiguousarray(q_pos, dtype=np.int32)
+        S = np.empty((T, max_blocks), np.float64)
+        sc = None if kidx_scale is None else np.ascontiguousarray(kidx_scale, dtype=np.float32)
+        self.lib.oracle_index_scores(_ptr(q), _ptr(w), _ptr(q_seq), _ptr(q_pos), T, Hi, _ptr(kidx),
+                                     kidx_fmt, _ptr(sc), kidx.shape[1] * 64,
+                                     0 if sc is None else sc.shape[1], m, max_blocks, _ptr(S))
+        return S
+
+    def topk(self, S, q_pos, m, k):
+        S = np.ascontiguousarray(S, dtype=np.float64)
+        T, max_blocks = S.shape
+        q_pos = np.ascontiguousarray(q_pos, dtype=np.int32)
+        idx = np.empty((T, k), np.int32)
+        sc = np.empty((T, k), np.float64)
+        self.lib.oracle_topk(_ptr(S), _ptr(q_pos), T, m, max_blocks, k, _ptr(idx), _ptr(sc))
+        return idx, sc
+
+    def sparse_attend(self, q, q_seq, q_pos, comp, raw, m, idx, W, scale):
+        """q uint16 [T][H][128]; comp uint16 [B][N][128]; raw uint16 [B][L][128];
+        idx int32 [T][k].  Returns out float64 [T][H][128], lse float64 [T][H]."""
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        T, H, _ = q.shape
+        comp = np.ascontiguousarray(comp, dtype=np.uint16)
+        raw = np.ascontiguousarray(raw, dtype=np.uint16)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        k = idx.shape[1]
+        out = np.empty((T, H, 128), np.float64)
+        lse = np.empty((T, H), np.float64)
+        self.lib.oracle_sparse_attend(_ptr(q), _ptr(np.ascontiguousarray(q_seq, dtype=np.int32)),
+                                      _ptr(np.ascontiguousarray(q_pos, dtype=np.int32)), T, H,
+                                      _ptr(comp), comp.shape[1] * 128, _ptr(raw), raw.shape[1] * 128,
+                                      m, _ptr(idx), k, W, scale, _ptr(out), _ptr(lse))
+        return out, lse
+
+    def hca_attend(self, q, q_seq, q_pos, comp, raw, m, W, scale):
+        q = np.ascontiguousarray(q, dtype=np.uint16)
+        T, H, _ = q.shape
+        comp = np.ascontiguousarray(comp, dtype=np.uint16)
+        raw = np.ascontiguousarray(raw, dtype=np.uint16)
+        out = np.empty((T, H, 128), np.float64)
+        lse = np.empty((T, H), np.float64)
+        self.lib.oracle_hca_attend(_ptr(q), _ptr(np.ascontiguousarray(q_seq, dtype=np.int32)),
+                                   _ptr(np.ascontiguousarray(q_pos, dtype=np.int32)), T, H,
+                                   _ptr(comp), comp.shape[1] * 128, _ptr(raw), raw.shape[1] * 128,
+                                   m, W, scale, _ptr(out), _ptr(lse))
+        return out, lse
+
+
+_DEFAULT = None
+
+
+def get(plant: int = 0) -> Oracle:
+    """The shared oracle handle (plant 0), or a fresh planted build."""
+    global _DEFAULT
+    if plant:
+        return Oracle(plant)
+    if _DEFAULT is None:
+        _DEFAULT = Oracle(0)
+    return _DEFAULT

@@ -1,0 +1,443 @@
+/*
+ * oracle.c -- plain, slow, double-precision CPU oracle for CSA / HCA.
+ *
+ * TEST INFRASTRUCTURE ONLY: see oracle.h.  No blocking, fusion or
+ * reordering beyond the definitions; loops follow the statement of the
+ * method (DeepSeek-V4 summary, b-lab.team, "Core Methodological
+ * Innovations", 1. Hybrid Attention Architecture, CSA and HCA bullets).
+ *
+ * ORACLE_PLANT: when compiled with -DORACLE_PLANT=n (n > 0), one deliberate
+ * mistake is planted so that the pin tests can show they catch it.  The
+ * shipped build uses ORACLE_PLANT=0 (no mistake).
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#ifndef ORACLE_PLANT
+#define ORACLE_PLANT 0
+#endif
+#define PLANT(n) (ORACLE_PLANT == (n))
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ */
+/* number formats                                                       */
+/* ------------------------------------------------------------------ */
+
+double oracle_bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round x to the nearest bf16 (8 significant bits, exponent range of
+ * fp32), ties to even, straight from double. */
+uint16_t oracle_double_to_bf16(double x) {
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    double r;
+    if (a == 0.0) return sign;
+    if (a < ldexp(1.0, -126)) {
+        /* subnormal range: fixed quantum 2^-133 */
+        r = rint(a / ldexp(1.0, -133)) * ldexp(1.0, -133);
+    } else {
+        int e;
+        double f = frexp(a, &e);         /* a = f * 2^e, f in [0.5, 1) */
+        double s = rint(ldexp(f, 8));    /* 8 significant bits, RNE */
+        r = ldexp(s, e - 8);
+    }
+    /* largest finite bf16 is (2 - 2^-7) * 2^127; past the rounding
+     * midpoint it becomes infinity */
+    if (r > ldexp(2.0 - ldexp(1.0, -7), 127)) return (uint16_t)(sign | 0x7F80);
+    float f32 = (float)r; /* exact: r has <= 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f32, 4);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFF));
+}
+
+/* OCP OFP8 E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits.
+ * Exponent field 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN;
+ * largest finite value 1.75 * 2^8 = 448. */
+double oracle_e4m3_to_double(uint8_t c) {
+    int s = (c >> 7) & 1, e = (c >> 3) & 15, mt = c & 7;
+    double v;
+    if (e == 15 && mt == 7) return NAN;
+    if (e == 0) v = ldexp((double)mt / 8.0, -6);
+    else v = ldexp(1.0 + (double)mt / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* Nearest E4M3 value to v, ties to even mantissa, magnitudes beyond 448
+ * clamp to 448 (saturating, finite).  NaN maps to 0x7F. */
+uint8_t oracle_float_to_e4m3_satfinite(float v) {
+    if (isnan(v)) return 0x7F;
+    uint8_t sign = signbit(v) ? 0x80 : 0;
+    double a = fabs((double)v);
+    double r;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal quantum 2^-9 */
+        double q = ldexp(1.0, -9);
+#if ORACLE_PLANT == 9
+        r = floor(a / q) * q; /* planted: truncation instead of RNE */
+#else
+        r = rint(a / q) * q;
+#endif
+    } else {
+        int e;
+        double f = frexp(a, &e);   /* a = f * 2^e */
+        double q = ldexp(1.0, e - 4);  /* 4 significant bits */
+#if ORACLE_PLANT == 9
+        r = floor(a / q) * q;
+#else
+        r = rint(a / q) * q;
+#endif
+    }
+    if (r > 448.0) r = 448.0;
+    if (r == 0.0) return sign;
+    int e;
+    double f = frexp(r, &e);       /* r = f * 2^e, f in [0.5, 1) */
+    int ebits = e - 1 + 7;         /* r = 1.x * 2^(e-1) */
+    uint8_t code;
+    if (ebits <= 0) {
+        /* subnormal: r = mt/8 * 2^-6 */
+        int mt = (int)lrint(r / ldexp(1.0, -9));
+        code = (uint8_t)mt;
+    } else {
+        int mt = (int)lrint((ldexp(f, 1) - 1.0) * 8.0);
+        code = (uint8_t)((ebits << 3) | mt);
+    }
+    return (uint8_t)(sign | code);
+}
+
+/* ------------------------------------------------------------------ */
+/* compression (CSA: m; HCA: m')                                        */
+/* ------------------------------------------------------------------ */
+
+/* Reading: "combining adjacent entries" is a fixed weighted sum of the m
+ * rows of a block, with per-position, per-channel weights normalised by a
+ * softmax over the m positions of each channel. */
+void oracle_pool_weights(const float* z, int m, int d, double* a) {
+#if ORACLE_PLANT == 2
+    /* planted: softmax taken over the channels instead of the positions */
+    for (int i = 0; i < m; ++i) {
+        double mx = -INFINITY, sum = 0.0;
+        for (int c = 0; c < d; ++c) if (z[i * d + c] > mx) mx = z[i * d + c];
+        for (int c = 0; c < d; ++c) sum += exp((double)z[i * d + c] - mx);
+        for (int c = 0; c < d; ++c) a[i * d + c] = exp((double)z[i * d + c] - mx) / sum;
+    }
+#else
+    for (int c = 0; c < d; ++c) {
+        double mx = -INFINITY;
+        for (int i = 0; i < m; ++i)
+            if (z[i * d + c] > mx) mx = z[i * d + c];
+        double sum = 0.0;
+        for (int i = 0; i < m; ++i) sum += exp((double)z[i * d + c] - mx);
+        for (int i = 0; i < m; ++i) a[i * d + c] = exp((double)z[i * d + c] - mx) / sum;
+    }
+#endif
+}
+
+void oracle_compress(const uint16_t* raw, int64_t raw_seq_stride,
+                     const int32_t* lens, int B, int d, int m,
+                     const float* z, int blk_lo, int blk_hi,
+                     int out_fmt, void* out, int64_t out_seq_stride,
+                     float* out_scale, int64_t scale_seq_stride) {
+    double* a = (double*)malloc(sizeof(double) * (size_t)m * d);
+    oracle_pool_weights(z, m, d, a);
+    double* row = (double*)malloc(sizeof(double) * d);
+    uint16_t* rb = (uint16_t*)malloc(sizeof(uint16_t) * d);
+    for (int b = 0; b < B; ++b) {
+        /* Reading: a trailing partial block (fewer than m rows) is not
+         * compressed; those tokens are reached only through the window. */
+        int nblk = lens[b] / m;
+        int lo, hi;
+        if (blk_lo >= 0) { lo = blk_lo; hi = blk_hi < nblk ? blk_hi : nblk; }
+        else { lo = nblk - blk_hi; if (lo < 0) lo = 0; hi = nblk; }
+        for (int j = lo; j < hi; ++j) {
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int i = 0; i < m; ++i) {
+#if ORACLE_PLANT == 1
+                    int64_t srow = (int64_t)j * m + i + 1; /* planted: off by one */
+#else
+                    int64_t srow = (int64_t)j * m + i;
+#endif
+                    acc += a[i * d + c] *
+                           oracle_bf16_to_double(raw[b * raw_seq_stride + srow * d + c]);
+                }
+                row[c] = acc;
+                rb[c] = oracle_double_to_bf16(acc);
+            }
+            if (out_fmt == 0) {
+                uint16_t* o = (uint16_t*)out + b * out_seq_stride + (int64_t)j * d;
+                memcpy(o, rb, sizeof(uint16_t) * d);
+            } else {
+                /* FP8 reading: quantise the bf16 row with one fp32 scale
+                 * per row, s = amax / 448 (s = 1 for an all-zero row). */
+                float amax = 0.0f;
+                for (int c = 0; c < d; ++c) {
+                    float v = fabsf((float)oracle_bf16_to_double(rb[c]));
+                    if (v > amax) amax = v;
+                }
+                float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+                uint8_t* o = (uint8_t*)out + b * out_seq_stride + (int64_t)j * d;
+                for (int c = 0; c < d; ++c) {
+                    float v = (float)oracle_bf16_to_double(rb[c]) / s;
+                    o[c] = oracle_float_to_e4m3_satfinite(v);
+                }
+                out_scale[b * scale_seq_stride + j] = s;
+            }
+        }
+    }
+    free(rb);
+    free(row);
+    free(a);
+}
+
+/* ------------------------------------------------------------------ */
+/* lightning indexer                                                    */
+/* ------------------------------------------------------------------ */
+
+/* The indexer query is a low-rank projection of the hidden state h_t:
+ * h -> u (rank r) -> q_h (64 per head).  Reading: the per-head weights
+ * w_h are a linear function of the same hidden state, w = W_w h. */
+void oracle_index_query(const uint16_t* h, int T, int D, int r, int Hi,
+                        const uint16_t* W_dq, const uint16_t* W_uq,
+                        const uint16_t* W_w, double* q_out, double* w_out) {
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        double* u = (double*)malloc(sizeof(double) * r);
+        const uint16_t* ht = h + (int64_t)t * D;
+        for (int i = 0; i < r; ++i) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += oracle_bf16_to_double(W_dq[(int64_t)i * D + c]) *
+                       oracle_bf16_to_double(ht[c]);
+            u[i] = acc;
+        }
+        for (int o = 0; o < Hi * 64; ++o) {
+            double acc = 0.0;
+            for (int i = 0; i < r; ++i)
+                acc += oracle_bf16_to_double(W_uq[(int64_t)o * r + i]) * u[i];
+            q_out[(int64_t)t * Hi * 64 + o] = acc;
+        }
+        for (int hh = 0; hh < Hi; ++hh) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c)
+                acc += oracle_bf16_to_double(W_w[(int64_t)hh * D + c]) *
+                       oracle_bf16_to_double(ht[c]);
+            w_out[(int64_t)t * Hi + hh] = acc;
+        }
+        free(u);
+    }
+}
+
+/* Causal visibility: compressed block j covers raw tokens [j m, j m + m);
+ * it is visible to a query at position p iff its last token j m + m - 1
+ * <= p, i.e. j < (p + 1) / m. */
+static int visible_blocks(int p, int m) {
+#if ORACLE_PLANT == 8
+    return p / m; /* planted: off by one in the visibility rule */
+#else
+    return (p + 1) / m;
+#endif
+}
+
+/* Score of one compressed block: sum over indexer heads of the head
+ * weight times the ReLU of the query-key dot product.  For FP8 keys the
+ * row scale multiplies the head sum (exact for s > 0, since
+ * ReLU(s x) = s ReLU(x)). */
+void oracle_index_scores(const double* q, const double* w,
+                         const int32_t* q_seq, const int32_t* q_pos, int T,
+                         int Hi, const void* kidx, int kidx_fmt,
+                         const float* kidx_scale, int64_t kidx_seq_stride,
+                         int64_t scale_seq_stride, int m, int max_blocks,
+                         double* S_out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        int b = q_seq[t];
+        int V = visible_blocks(q_pos[t], m);
+        double* S = S_out + (int64_t)t * max_blocks;
+        double key[64];
+        for (int j = 0; j < max_blocks; ++j) {
+            if (j >= V) { S[j] = NAN; continue; }
+            double s = 1.0;
+            if (kidx_fmt == 0) {
+                const uint16_t* kr = (const uint16_t*)kidx + b * kidx_seq_stride + (int64_t)j * 64;
+                for (int c = 0; c < 64; ++c) key[c] = oracle_bf16_to_double(kr[c]);
+            } else {
+                const uint8_t* kr = (const uint8_t*)kidx + b * kidx_seq_stride + (int64_t)j * 64;
+                for (int c = 0; c < 64; ++c) key[c] = oracle_e4m3_to_double(kr[c]);
+                s = (double)kidx_scale[b * scale_seq_stride + j];
+            }
+            double acc = 0.0;
+            for (int hh = 0; hh < Hi; ++hh) {
+                const double* qh = q + ((int64_t)t * Hi + hh) * 64;
+                double dot = 0.0;
+                for (int c = 0; c < 64; ++c) dot += qh[c] * key[c];
+#if ORACLE_PLANT == 3
+                double act = dot;                     /* planted: ReLU dropped */
+#else
+                double act = dot > 0.0 ? dot : 0.0;
+#endif
+#if ORACLE_PLANT == 4
+                acc += act;                           /* planted: head weight dropped */
+#else
+                acc += w[(int64_t)t * Hi + hh] * act;
+#endif
+            }
+            S[j] = s * acc;
+        }
+    }
+}
+
+typedef struct { double s; int32_t j; } scored_t;
+
+/* Score descending, then block index ascending (a total order, so the
+ * unstable qsort still gives one answer). */
+static int cmp_scored(const void* x, const void* y) {
+    const scored_t* a = (const scored_t*)x;
+    const scored_t* b = (const scored_t*)y;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+#if ORACLE_PLANT == 5
+    return (a->j > b->j) ? -1 : (a->j < b->j); /* planted: ties by index descending */
+#else
+    return (a->j < b->j) ? -1 : (a->j > b->j);
+#endif
+}
+
+void oracle_topk(const double* S, const int32_t* q_pos, int T, int m,
+                 int max_blocks, int k, int32_t* out_idx, double* out_score) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        int V = visible_blocks(q_pos[t], m);
+        if (V > max_blocks) V = max_blocks;
+        scored_t* v = (scored_t*)malloc(sizeof(scored_t) * (V > 0 ? V : 1));
+        for (int j = 0; j < V; ++j) { v[j].s = S[(int64_t)t * max_blocks + j]; v[j].j = j; }
+        qsort(v, (size_t)V, sizeof(scored_t), cmp_scored);
+        for (int i = 0; i < k; ++i) {
+            if (i < V) {
+                out_idx[(int64_t)t * k + i] = v[i].j;
+                if (out_score) out_score[(int64_t)t * k + i] = v[i].s;
+            } else {
+                out_idx[(int64_t)t * k + i] = -1;
+                if (out_score) out_score[(int64_t)t * k + i] = NAN;
+            }
+        }
+        free(v);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* attention over an explicit set of latent rows                        */
+/* ------------------------------------------------------------------ */
+
+/* o_h = sum_e softmax_e(scale * q_h . x_e) x_e over the rows rows[0..n),
+ * with K = V = the latent row (reading: the pages name no separate value
+ * projection), two passes in double. */
+static void attend_rows(const uint16_t* qt, int H, const uint16_t** rows, int n,
+                        double scale, double* out, double* lse) {
+    double* z = (double*)malloc(sizeof(double) * (n > 0 ? n : 1));
+    for (int hh = 0; hh < H; ++hh) {
+        const uint16_t* qh = qt + (int64_t)hh * 128;
+        double* o = out + (int64_t)hh * 128;
+        for (int c = 0; c < 128; ++c) o[c] = 0.0;
+        if (n == 0) { lse[hh] = -INFINITY; continue; }
+        double mx = -INFINITY;
+        for (int e = 0; e < n; ++e) {
+            double dot = 0.0;
+            for (int c = 0; c < 128; ++c)
+                dot += oracle_bf16_to_double(qh[c]) * oracle_bf16_to_double(rows[e][c]);
+#if ORACLE_PLANT == 7
+            z[e] = dot;                 /* planted: softmax scale dropped */
+#else
+            z[e] = scale * dot;
+#endif
+            if (z[e] > mx) mx = z[e];
+        }
+        double sum = 0.0;
+        for (int e = 0; e < n; ++e) sum += exp(z[e] - mx);
+        for (int e = 0; e < n; ++e) {
+            double p = exp(z[e] - mx) / sum;
+            for (int c = 0; c < 128; ++c) o[c] += p * oracle_bf16_to_double(rows[e][c]);
+        }
+        lse[hh] = mx + log(sum);
+    }
+    free(z);
+}
+
+/* Sliding window: the raw rows s with p - W < s <= p and s >= 0. */
+static int window_rows(const uint16_t* raw_b, int p, int W, const uint16_t** rows) {
+    int n = 0;
+#if ORACLE_PLANT == 6
+    for (int s = p - W + 1; s < p; ++s) { /* planted: query's own row dropped */
+#else
+    for (int s = p - W + 1; s <= p; ++s) {
+#endif
+        if (s < 0) continue;
+        rows[n++] = raw_b + (int64_t)s * 128;
+    }
+    return n;
+}
+
+void oracle_sparse_attend(const uint16_t* q, const int32_t* q_seq,
+                          const int32_t* q_pos, int T, int H,
+                          const uint16_t* comp, int64_t comp_seq_stride,
+                          const uint16_t* raw, int64_t raw_seq_stride, int m,
+                          const int32_t* idx, int k, int W, double scale,
+                          double* out, double* lse) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        int b = q_seq[t], p = q_pos[t];
+        int V = visible_blocks(p, m);
+        const uint16_t** rows = (const uint16_t**)malloc(sizeof(uint16_t*) * (size_t)(k + W + 1));
+        int n = 0;
+        for (int i = 0; i < k; ++i) {
+            int j = idx[(int64_t)t * k + i];
+            if (j < 0 || j >= V) continue;   /* padding or invalid: skipped */
+            rows[n++] = comp + b * comp_seq_stride + (int64_t)j * 128;
+        }
+        /* Reading: a compressed block that also lies inside the window is
+         * attended in both forms (no de-duplication). */
+        n += window_rows(raw + b * raw_seq_stride, p, W, rows + n);
+        attend_rows(q + (int64_t)t * H * 128, H, rows, n, scale,
+                    out + (int64_t)t * H * 128, lse + (int64_t)t * H);
+        free(rows);
+    }
+}
+
+void oracle_hca_attend(const uint16_t* q, const int32_t* q_seq,
+                       const int32_t* q_pos, int T, int H,
+                       const uint16_t* comp, int64_t comp_seq_stride,
+                       const uint16_t* raw, int64_t raw_seq_stride, int m,
+                       int W, double scale, double* out, double* lse) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; ++t) {
+        int b = q_seq[t], p = q_pos[t];
+        int V = visible_blocks(p, m);
+        const uint16_t** rows = (const uint16_t**)malloc(sizeof(uint16_t*) * (size_t)(V + W + 1));
+        int n = 0;
+        for (int j = 0; j < V; ++j) rows[n++] = comp + b * comp_seq_stride + (int64_t)j * 128;
+#if ORACLE_PLANT != 10
+        n += window_rows(raw + b * raw_seq_stride, p, W, rows + n);
+#endif
+        attend_rows(q + (int64_t)t * H * 128, H, rows, n, scale,
+                    out + (int64_t)t * H * 128, lse + (int64_t)t * H);
+        free(rows);
+    }
+}

@@ -1,0 +1,119 @@
+/*
+ * oracle.h -- plain, slow CPU oracle for the CSA / HCA hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link,
+ * load or call this code: only tests/, the package smoke check and the
+ * bench's cpu_baseline / reference leg use it.  It shares no code, header,
+ * table or constant with the CUDA library under long_context_sparse_03_b200/.
+ *
+ * Sources.  The method is stated in two sentences of the page
+ * "DeepSeek-V4" summary on b-lab.team, section "Core Methodological
+ * Innovations", item 1 "Hybrid Attention Architecture (CSA and HCA)":
+ *   - CSA bullet: the KV cache is compressed by a factor m by combining
+ *     adjacent entries; a "Lightning Indexer" scores compressed blocks from
+ *     low-rank projections of the query hidden state h_t and the top-k
+ *     blocks are attended.
+ *   - HCA bullet: compression by m' >> m with dense attention over what
+ *     remains; both are supplemented by a sliding window of local entries.
+ * Everything the pages leave open (pooling form, score formula, window
+ * rule, number formats) is fixed by the readings listed beside each
+ * function below; they are the plainest ones the statement supports.
+ *
+ * Arithmetic: every floating-point result is accumulated in double from the
+ * bf16 / fp32 inputs.  The only fp32 steps are the FP8 quantisation
+ * decisions (scale and code), which the oracle takes in fp32 so that an
+ * integer code is decided in the same precision on both sides.
+ *
+ * Parity status: every function here is pinned by tests/test_oracle_pins.py
+ * (closed forms, special cases, brute force on tiny inputs).  The absolute
+ * values at full workload sizes are pinned only through those identities.
+ */
+#ifndef CSA_ORACLE_H
+#define CSA_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* bf16 <-> double.  The encoder rounds a double straight to the nearest
+ * bf16 (ties to even), never through float, to avoid double rounding. */
+double   oracle_bf16_to_double(uint16_t b);
+uint16_t oracle_double_to_bf16(double x);
+
+/* OCP OFP8 E4M3 (bias 7, max 448, no infinities, 0x7F/0xFF = NaN). */
+double  oracle_e4m3_to_double(uint8_t c);
+uint8_t oracle_float_to_e4m3_satfinite(float v);
+
+/* Pooling weights a[i][c] = softmax over i of logits z[i][c], in double. */
+void oracle_pool_weights(const float* z, int m, int d, double* a_out);
+
+/* Compress adjacent rows by m (CSA) or m' (HCA):
+ *   C[b][j][c] = sum_{i<m} a[i][c] * X[b][j*m+i][c],  a = softmax_i(z[:,c])
+ * for blocks j in the requested range that are complete (j*m+m <= lens[b]).
+ * blk_lo >= 0: absolute range [blk_lo, blk_hi).  blk_lo < 0: the last
+ * blk_hi complete blocks of each sequence.
+ * out_fmt 0: bf16 rows.  out_fmt 1: FP8 E4M3 rows + one fp32 scale per row
+ * (the bf16 row is formed first, then s = amax/448 in fp32 (1 if amax == 0)
+ * and code = e4m3_rn_satfinite(x / s) in fp32).
+ * Strides are in elements (rows * d for the caches, rows for scales). */
+void oracle_compress(const uint16_t* raw, int64_t raw_seq_stride,
+                     const int32_t* lens, int B, int d, int m,
+                     const float* z, int blk_lo, int blk_hi,
+                     int out_fmt, void* out, int64_t out_seq_stride,
+                     float* out_scale, int64_t scale_seq_stride);
+
+/* Indexer query: u = W_dq h (rank r), q_h = W_uq[h] u (64 each), w = W_w h.
+ * h [T][D], W_dq [r][D], W_uq [Hi*64][r], W_w [Hi][D], all bf16.
+ * q_out [T][Hi][64], w_out [T][Hi] in double. */
+void oracle_index_query(const uint16_t* h, int T, int D, int r, int Hi,
+                        const uint16_t* W_dq, const uint16_t* W_uq,
+                        const uint16_t* W_w, double* q_out, double* w_out);
+
+/* Indexer scores S[t][j] = sum_h w_h * max(0, q_h . k_j)  (times s_j for
+ * FP8 keys) for the blocks visible to query t: j < V(t) = (q_pos+1) / m.
+ * Entries j >= V(t) (up to max_blocks) are set to NaN.
+ * kidx_fmt 0: bf16 keys [B][stride][64]; 1: E4M3 keys + fp32 scale. */
+void oracle_index_scores(const double* q, const double* w,
+                         const int32_t* q_seq, const int32_t* q_pos, int T,
+                         int Hi, const void* kidx, int kidx_fmt,
+                         const float* kidx_scale, int64_t kidx_seq_stride,
+                         int64_t scale_seq_stride, int m, int max_blocks,
+                         double* S_out);
+
+/* Per-query top-k over the visible scores: order by score descending, then
+ * block index ascending; the first min(k, V(t)) are written, the rest of
+ * the row is -1 (score NaN). */
+void oracle_topk(const double* S, const int32_t* q_pos, int T, int m,
+                 int max_blocks, int k, int32_t* out_idx, double* out_score);
+
+/* CSA sparse attention.  For query t of sequence b = q_seq[t] at position
+ * p = q_pos[t], the attended set is
+ *   E = { C[b][j] : j = idx[t][i], 0 <= j < V(t) }  (idx < 0 skipped)
+ *     + { X[b][s] : p - W < s <= p, s >= 0 }          (raw window)
+ * with K = V = the 128-d latent row; o_h = sum_e softmax_e(scale q_h.x_e) x_e
+ * and lse_h = log sum_e exp(scale q_h.x_e).  Empty E gives o = 0,
+ * lse = -inf.  q [T][H][128] bf16; out [T][H][128], lse [T][H] double. */
+void oracle_sparse_attend(const uint16_t* q, const int32_t* q_seq,
+                          const int32_t* q_pos, int T, int H,
+                          const uint16_t* comp, int64_t comp_seq_stride,
+                          const uint16_t* raw, int64_t raw_seq_stride, int m,
+                          const int32_t* idx, int k, int W, double scale,
+                          double* out, double* lse);
+
+/* HCA dense attention: E = all visible compressed rows j < V(t) (pooled by
+ * m = m') plus the same raw window. */
+void oracle_hca_attend(const uint16_t* q, const int32_t* q_seq,
+                       const int32_t* q_pos, int T, int H,
+                       const uint16_t* comp, int64_t comp_seq_stride,
+                       const uint16_t* raw, int64_t raw_seq_stride, int m,
+                       int W, double scale, double* out, double* lse);
+
+/* Number of OpenMP threads the oracle runs with (1 without OpenMP). */
+int oracle_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

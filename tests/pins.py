@@ -1,0 +1,456 @@
+"""Pins for the CPU oracle: checks that do not restate the oracle's loops.
+
+Each pin fixes one part of the oracle against something other than itself:
+a library routine for a special case (numpy / scipy / torch), a closed form,
+an invariant, the OCP E4M3 table, or brute force on tiny inputs.  They are
+plain functions taking an oracle handle so that ``test_oracle_pins.py`` can
+run them on the shipped oracle and on builds with a planted mistake.
+
+Sources of the definitions: DeepSeek-V4 summary page (b-lab.team), "Core
+Methodological Innovations", 1. Hybrid Attention Architecture -- the CSA
+bullet (compress by m, lightning indexer over low-rank projections of h_t,
+top-k blocks, sparse attention) and the HCA bullet (compress by m' >> m,
+dense attention, sliding window of local entries).
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import scipy.special
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------- helpers
+def bf16_bits_to_f64(u):
+    u = np.asarray(u, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def rand_bf16(rng, shape, scale=1.0):
+    x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32) * scale)
+    return x.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_neighbours_ok(x, b):
+    """b (bf16 bits) is a nearest bf16 to x (float64), ties to even."""
+    x = np.asarray(x, np.float64).ravel()
+    b = np.asarray(b, np.uint16).ravel()
+    v = bf16_bits_to_f64(b)
+    for dlt in (1, -1):
+        nb = (b.astype(np.int32) + dlt).astype(np.uint16)
+        nv = bf16_bits_to_f64(nb)
+        ok = np.isfinite(nv)
+        err_b = np.abs(x - v)
+        err_n = np.abs(x - nv)
+        bad = ok & ((err_n < err_b) | ((err_n == err_b) & ((b & 1) == 1)))
+        assert not bad.any(), f"not nearest-even bf16 at {np.nonzero(bad)[0][:5]}"
+
+
+def causal_attention(q, rows, scale):
+    """Full softmax attention of q [H][128] over rows [n][128] via scipy."""
+    z = scale * (q @ rows.T)
+    p = scipy.special.softmax(z, axis=1)
+    return p @ rows, scipy.special.logsumexp(z, axis=1)
+
+
+# ---------------------------------------------------------------- formats
+def pin_bf16_encoder(o):
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(2000) * 10.0 ** rng.integers(-30, 30, 2000),
+                        [0.0, -0.0, 1.0, -3.5, 1e-40, 3.3e38]])
+    b = o.to_bf16(x)
+    bf16_neighbours_ok(x, b)
+    # values exact in fp32 must agree with torch's fp32 -> bf16 (RNE) cast
+    x32 = x.astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(x32.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(o.to_bf16(x32), ref)
+
+
+def pin_e4m3_table(o):
+    rows = []
+    with open(os.path.join(GOLDEN, "e4m3_ocp.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                v, c = line.split()[:2]
+                rows.append((float(v), int(c, 16)))
+    vals = np.array([r[0] for r in rows], np.float32)
+    codes = o.e4m3_encode(vals)
+    assert codes.tolist() == [r[1] for r in rows], list(zip(vals.tolist(), codes.tolist()))
+    # decoding: every code against torch's float8_e4m3fn
+    allc = np.arange(256, dtype=np.uint8)
+    dec = o.e4m3_decode(allc)
+    ref = torch.from_numpy(allc).view(torch.float8_e4m3fn).float().double().numpy()
+    same = (dec == ref) | (np.isnan(dec) & np.isnan(ref))
+    assert same.all()
+
+
+def pin_e4m3_encoder_vs_torch(o):
+    rng = np.random.default_rng(2)
+    v = (rng.standard_normal(4000) * 2.0 ** rng.integers(-12, 9, 4000)).astype(np.float32)
+    v = v[np.abs(v) <= 464.0]
+    c = o.e4m3_encode(v)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(c, ref)
+
+
+# ---------------------------------------------------------------- compress
+def _compress_case(rng, B=2, L=37, d=128, m=4):
+    raw = rand_bf16(rng, (B, L, d))
+    lens = np.array([L, L - 5][:B], np.int32)
+    return raw, lens
+
+
+def pin_compress_one_hot(o):
+    """One-hot pooling weights reproduce strided subsampling exactly."""
+    rng = np.random.default_rng(3)
+    for m, i0, d in ((4, 0, 128), (4, 3, 128), (8, 5, 64), (128, 77, 128)):
+        L = m * 5 + 1
+        raw, lens = _compress_case(rng, B=2, L=L, d=d, m=m)
+        z = np.full((m, d), -np.inf, np.float32)
+        z[i0] = 0.0
+        out, _ = o.compress(raw, lens, z, 0, 1 << 30)
+        for b in range(2):
+            nb = lens[b] // m
+            assert np.array_equal(out[b, :nb], raw[b, i0:nb * m:m]), (m, i0, b)
+
+
+def pin_compress_mean(o):
+    """Equal logits give the block mean, rounded to the nearest bf16."""
+    rng = np.random.default_rng(4)
+    m, d = 4, 128
+    raw, lens = _compress_case(rng, B=2, L=41, d=d, m=m)
+    z = np.full((m, d), 0.37, np.float32)
+    out, _ = o.compress(raw, lens, z, 0, 1 << 30)
+    for b in range(2):
+        nb = lens[b] // m
+        x = bf16_bits_to_f64(raw[b, :nb * m]).reshape(nb, m, d)
+        mean = x.sum(axis=1) / m          # exact in float64 for these values
+        bf16_neighbours_ok(mean, out[b, :nb])
+
+
+def pin_compress_identity(o):
+    """m = 1 is the identity; m identical rows give that row back."""
+    rng = np.random.default_rng(5)
+    raw, lens = _compress_case(rng, B=1, L=9, d=128, m=1)
+    z = rng.standard_normal((1, 128)).astype(np.float32)
+    out, _ = o.compress(raw, lens, z, 0, 1 << 30)
+    assert np.array_equal(out[0, :9], raw[0, :9])
+    m = 8
+    row = rand_bf16(rng, (1, 1, 128))
+    raw2 = np.repeat(row, 3 * m, axis=1)
+    z = rng.standard_normal((m, 128)).astype(np.float32) * 3
+    out, _ = o.compress(raw2, np.array([3 * m], np.int32), z, 0, 1 << 30)
+    assert np.array_equal(out[0, :3], np.repeat(row[0], 3, axis=0))
+
+
+def pin_pool_weights(o):
+    """The weights are a softmax over the m positions of each channel."""
+    rng = np.random.default_rng(6)
+    z = rng.standard_normal((4, 128)).astype(np.float32)
+    a = o.pool_weights(z)
+    assert np.allclose(a, scipy.special.softmax(z.astype(np.float64), axis=0), rtol=1e-14, atol=0)
+
+
+def pin_compress_ranges(o):
+    """Partial trailing blocks are not compressed; the relative range only
+    touches the newest complete blocks."""
+    rng = np.random.default_rng(7)
+    m, d = 4, 64
+    raw = rand_bf16(rng, (2, 30, d))
+    lens = np.array([30, 17], np.int32)          # 7 and 4 complete blocks
+    z = rng.standard_normal((m, d)).astype(np.float32)
+    canary = np.uint16(0x7FA1)
+    out = np.full((2, 8, d), canary, np.uint16)
+    o.compress(raw, lens, z, 0, 1 << 30, out=out)
+    assert (out[0, 7] == canary).all() and (out[1, 4:] == canary).all()
+    assert not (out[0, :7] == canary).any() and not (out[1, :4] == canary).any()
+    out2 = np.full((2, 8, d), canary, np.uint16)
+    o.compress(raw, lens, z, -1, 1, out=out2)
+    assert np.array_equal(out2[0, 6], out[0, 6]) and np.array_equal(out2[1, 3], out[1, 3])
+    out2[0, 6] = canary
+    out2[1, 3] = canary
+    assert (out2 == canary).all()
+    # the block ending exactly at the last raw row is complete
+    out3, _ = o.compress(raw[:, :16], np.array([16, 15], np.int32), z, 0, 1 << 30)
+    z1 = np.full((m, d), -np.inf, np.float32)
+    z1[m - 1] = 0
+    o3, _ = o.compress(raw[:, :16], np.array([16, 15], np.int32), z1, 0, 1 << 30)
+    assert np.array_equal(o3[0, 3], raw[0, 15])
+
+
+def pin_compress_fp8(o):
+    """E4M3 rows: with exact pooling (one-hot) the codes are the torch
+    E4M3 cast of bf16 / s, s = amax / 448 in fp32; the amax element maps to
+    +-448 and an all-zero row has s = 1."""
+    rng = np.random.default_rng(8)
+    m, d = 4, 64
+    raw = rand_bf16(rng, (2, 24, d))
+    raw[1, 8:12] = 0                               # block 2 of seq 1 is all zero
+    lens = np.array([24, 24], np.int32)
+    z = np.full((m, d), -np.inf, np.float32)
+    z[1] = 0.0
+    codes, scale = o.compress(raw, lens, z, 0, 1 << 30, out_fmt=1)
+    for b in range(2):
+        for j in range(6):
+            x = bf16_bits_to_f64(raw[b, j * m + 1]).astype(np.float32)
+            amax = np.float32(np.abs(x).max())
+            s = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+            assert scale[b, j] == s
+            ref = torch.from_numpy((x / s).astype(np.float32)).to(torch.float8_e4m3fn)
+            assert np.array_equal(codes[b, j], ref.view(torch.uint8).numpy()), (b, j)
+            if amax > 0:
+                assert (codes[b, j] & 0x7F).max() == 0x7E
+    assert scale[1, 2] == 1.0 and (codes[1, 2] == 0).all()
+
+
+# ---------------------------------------------------------------- indexer
+def pin_index_query(o):
+    """q = W_uq (W_dq h) per head and w = W_w h, against numpy matmuls."""
+    rng = np.random.default_rng(9)
+    T, D, r, Hi = 3, 96, 40, 5
+    h = rand_bf16(rng, (T, D))
+    W_dq = rand_bf16(rng, (r, D), D ** -0.5)
+    W_uq = rand_bf16(rng, (Hi * 64, r), r ** -0.5)
+    W_w = rand_bf16(rng, (Hi, D), D ** -0.5)
+    q, w = o.index_query(h, W_dq, W_uq, W_w)
+    hf, dq, uq, ww = (bf16_bits_to_f64(x) for x in (h, W_dq, W_uq, W_w))
+    u = hf @ dq.T
+    assert np.allclose(q, (u @ uq.T).reshape(T, Hi, 64), rtol=1e-12, atol=1e-12)
+    assert np.allclose(w, hf @ ww.T, rtol=1e-12, atol=1e-12)
+    # h -> 2h (exact in bf16) doubles both outputs exactly
+    h2 = torch.from_numpy(bf16_bits_to_f64(h).astype(np.float32) * 2).to(torch.bfloat16)
+    q2, w2 = o.index_query(h2.view(torch.int16).numpy().view(np.uint16), W_dq, W_uq, W_w)
+    assert np.array_equal(q2, 2 * q) and np.array_equal(w2, 2 * w)
+
+
+def _keys(rng, B, N):
+    return rand_bf16(rng, (B, N, 64))
+
+
+def pin_scores_closed_forms(o):
+    """Unit-vector keys give S_j = sum_h w_h max(0, q_h[c_j]); one head with
+    w = 1 gives max(0, q . k_j); keys with every dot negative score 0."""
+    rng = np.random.default_rng(10)
+    Hi, m = 3, 4
+    N = 64
+    cols = rng.integers(0, 64, N)
+    keys = np.zeros((1, N, 64), np.uint16)
+    keys[0, np.arange(N), cols] = 0x3F80                   # bf16 1.0
+    q = rng.standard_normal((1, Hi, 64))
+    w = rng.standard_normal((1, Hi))
+    S = o.index_scores(q, w, [0], [N * m - 1], keys, m, N)
+    ref = (w[0][:, None] * np.maximum(q[0][:, cols], 0)).sum(axis=0)
+    assert np.allclose(S[0], ref, rtol=1e-14, atol=1e-14)
+    k2 = _keys(rng, 1, N)
+    q1 = rng.standard_normal((1, 1, 64))
+    S1 = o.index_scores(q1, np.ones((1, 1)), [0], [N * m - 1], k2, m, N)
+    assert np.allclose(S1[0], np.maximum(bf16_bits_to_f64(k2[0]) @ q1[0, 0], 0), rtol=1e-13, atol=1e-13)
+    # all dots negative -> exactly zero whatever the weights
+    qn = -np.abs(rng.standard_normal((1, Hi, 64)))
+    kp = np.abs(bf16_bits_to_f64(k2[0])).astype(np.float32)
+    kp = torch.from_numpy(kp).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)[None]
+    S0 = o.index_scores(qn, w, [0], [N * m - 1], kp, m, N)
+    assert (S0 == 0).all()
+
+
+def pin_scores_brute(o):
+    """Brute force on tiny inputs: einsum over heads and dims; invisible
+    blocks are NaN and the visibility edge is exact."""
+    rng = np.random.default_rng(11)
+    B, N, Hi, m = 2, 12, 4, 4
+    keys = _keys(rng, B, N)
+    T = 4
+    q = rng.standard_normal((T, Hi, 64))
+    w = rng.standard_normal((T, Hi))
+    q_seq = np.array([0, 1, 1, 0], np.int32)
+    q_pos = np.array([47, 30, 31, 2], np.int32)              # V = 12, 7, 8, 0
+    S = o.index_scores(q, w, q_seq, q_pos, keys, m, N)
+    kf = bf16_bits_to_f64(keys)
+    for t in range(T):
+        V = (q_pos[t] + 1) // m
+        dots = np.einsum("hc,jc->hj", q[t], kf[q_seq[t], :N])
+        ref = (w[t][:, None] * np.maximum(dots, 0)).sum(0)
+        assert np.allclose(S[t, :V], ref[:V], rtol=1e-12, atol=1e-12)
+        assert np.isnan(S[t, V:]).all()
+
+
+def pin_scores_fp8_factoring(o):
+    """E4M3 keys: S = s_j * (score of the decoded codes), since
+    ReLU(s x) = s ReLU(x) for s > 0."""
+    rng = np.random.default_rng(12)
+    N, Hi, m = 16, 4, 4
+    codes = rng.integers(0, 256, (1, N, 64)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C                      # no NaN codes
+    scale = (rng.random((1, N)) * 3 + 0.1).astype(np.float32)
+    q = rng.standard_normal((1, Hi, 64))
+    w = rng.standard_normal((1, Hi))
+    S8 = o.index_scores(q, w, [0], [N * m - 1], codes, m, N, kidx_fmt=1, kidx_scale=scale)
+    dec = torch.from_numpy(codes).view(torch.float8_e4m3fn).float()          # library decode
+    kb = dec.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)    # exact in bf16
+    Sb = o.index_scores(q, w, [0], [N * m - 1], kb, m, N)
+    assert np.allclose(S8, Sb * scale.astype(np.float64), rtol=1e-13, atol=1e-13)
+
+
+def pin_topk_full_sort(o):
+    """Top-k equals a full sort by (score desc, index asc) on tiny inputs,
+    with injected ties, +-0 ties, k >= V padding."""
+    rng = np.random.default_rng(13)
+    T, N, m = 5, 40, 4
+    S = np.round(rng.standard_normal((T, N)) * 4) / 4                 # many ties
+    S[2, :10] = 0.0
+    S[2, 10:20] = -0.0
+    q_pos = np.array([159, 159, 159, 50, 3], np.int32)                # V = 40, 40, 40, 12, 1
+    for t in range(T):
+        S[t, (q_pos[t] + 1) // m:] = np.nan
+    for k in (1, 7, 12, 40, 45):
+        idx, sc = o.topk(S, q_pos, m, k)
+        for t in range(T):
+            V = (q_pos[t] + 1) // m
+            js = np.arange(V)
+            order = np.lexsort((js, -S[t, :V]))                       # by -S, then j
+            ref = order[:k]
+            n = min(k, V)
+            assert np.array_equal(idx[t, :n], ref[:n]), (k, t)
+            assert (idx[t, n:] == -1).all()
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(rng, B, L, N, H):
+    q = rand_bf16(rng, (B, H, 128))
+    comp = rand_bf16(rng, (B, N, 128))
+    raw = rand_bf16(rng, (B, L, 128))
+    return q, comp, raw
+
+
+def pin_attend_full_causal(o):
+    """m = 1, k = every visible block, W = 0: CSA is full causal softmax
+    attention over the raw rows (compressed rows = raw rows)."""
+    rng = np.random.default_rng(14)
+    B, L, H = 2, 50, 16
+    q, _, raw = _attn_case(rng, B, L, 1, H)
+    q_seq = np.array([0, 1], np.int32)
+    q_pos = np.array([49, 23], np.int32)
+    k = 50
+    idx = np.full((B, k), -1, np.int32)
+    for t in range(B):
+        idx[t, :q_pos[t] + 1] = rng.permutation(q_pos[t] + 1)
+    scale = 128 ** -0.5
+    out, lse = o.sparse_attend(q, q_seq, q_pos, raw, raw, 1, idx, 0, scale)
+    for t in range(B):
+        rows = bf16_bits_to_f64(raw[t, :q_pos[t] + 1])
+        ref, rl = causal_attention(bf16_bits_to_f64(q[t]), rows, scale)
+        assert np.allclose(out[t], ref, rtol=1e-12, atol=1e-12)
+        assert np.allclose(lse[t], rl, rtol=1e-12, atol=1e-12)
+
+
+def pin_attend_special_sets(o):
+    """k = 1, W = 0 returns the selected row; identical rows return that
+    row; permuting the index list changes nothing; -1 entries are skipped;
+    an empty set gives 0 and lse = -inf."""
+    rng = np.random.default_rng(15)
+    B, L, N, H, m = 1, 64, 16, 16, 4
+    q, comp, raw = _attn_case(rng, B, L, N, H)
+    scale = 128 ** -0.5
+    out, lse = o.sparse_attend(q, [0], [63], comp, raw, m, np.array([[5]], np.int32), 0, scale)
+    assert np.array_equal(out[0], np.repeat(bf16_bits_to_f64(comp[0, 5])[None], H, 0))
+    assert np.allclose(lse[0], scale * bf16_bits_to_f64(q[0]) @ bf16_bits_to_f64(comp[0, 5]), rtol=1e-13)
+    same = np.repeat(comp[:, :1], N, axis=1)
+    same_raw = np.repeat(comp[:, :1], L, axis=1)
+    idx = np.arange(8, dtype=np.int32)[None]
+    out, _ = o.sparse_attend(q, [0], [63], same, same_raw, m, idx, 4, scale)
+    assert np.allclose(out[0], np.repeat(bf16_bits_to_f64(same[0, 0])[None], H, 0), rtol=1e-14, atol=1e-14)
+    idx = np.array([[3, 9, 1, 14, -1, 7]], np.int32)
+    o1, l1 = o.sparse_attend(q, [0], [63], comp, raw, m, idx, 8, scale)
+    o2, l2 = o.sparse_attend(q, [0], [63], comp, raw, m, idx[:, [5, 4, 3, 2, 1, 0]], 8, scale)
+    o3, l3 = o.sparse_attend(q, [0], [63], comp, raw, m, np.array([[7, 14, 1, 9, 3]], np.int32), 8, scale)
+    assert np.allclose(o1, o2, rtol=1e-13, atol=1e-13) and np.allclose(o1, o3, rtol=1e-13, atol=1e-13)
+    assert np.allclose(l1, l3, rtol=1e-13)
+    # query at position 2 < m - 1 with no window: nothing is visible
+    oe, le = o.sparse_attend(q, [0], [2], comp, raw, m, np.array([[-1, -1]], np.int32), 0, scale)
+    assert (oe == 0).all() and np.isneginf(le).all()
+
+
+def pin_attend_window_no_dedup(o):
+    """With m = 1, k = every block and a window of W rows, each window row
+    appears twice in the attended set (closed form: softmax over the list
+    with those rows duplicated)."""
+    rng = np.random.default_rng(16)
+    L, H, W = 30, 16, 6
+    q, _, raw = _attn_case(rng, 1, L, 1, H)
+    p = 20
+    idx = np.arange(p + 1, dtype=np.int32)[None]
+    scale = 0.1
+    out, lse = o.sparse_attend(q, [0], [p], raw, raw, 1, idx, W, scale)
+    rows = bf16_bits_to_f64(raw[0])
+    lst = np.concatenate([rows[:p + 1], rows[p - W + 1:p + 1]])
+    ref, rl = causal_attention(bf16_bits_to_f64(q[0]), lst, scale)
+    assert np.allclose(out[0], ref, rtol=1e-12, atol=1e-12) and np.allclose(lse[0], rl, rtol=1e-12)
+    # window only (k = 0 selected): the last W raw rows, clipped at 0
+    out, lse = o.sparse_attend(q, [0], [3], raw, raw, 4, np.full((1, 1), -1, np.int32), W, scale)
+    ref, rl = causal_attention(bf16_bits_to_f64(q[0]), rows[:4], scale)
+    assert np.allclose(out[0], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_hca_equals_csa_all(o):
+    """HCA equals CSA with k = all visible blocks, and with m' = 1, W = 0
+    it is full causal attention."""
+    rng = np.random.default_rng(17)
+    B, L, H, m, W = 2, 700, 16, 128, 128
+    N = L // m
+    q, comp, raw = _attn_case(rng, B, L, N, H)
+    q_seq = np.array([0, 1], np.int32)
+    q_pos = np.array([699, 300], np.int32)
+    scale = 128 ** -0.5
+    oh, lh = o.hca_attend(q, q_seq, q_pos, comp, raw, m, W, scale)
+    idx = np.full((B, N), -1, np.int32)
+    for t in range(B):
+        V = (q_pos[t] + 1) // m
+        idx[t, :V] = np.arange(V)[::-1]
+    oc, lc = o.sparse_attend(q, q_seq, q_pos, comp, raw, m, idx, W, scale)
+    assert np.allclose(oh, oc, rtol=1e-13, atol=1e-13) and np.allclose(lh, lc, rtol=1e-13)
+    of, lf = o.hca_attend(q, q_seq, np.array([40, 9], np.int32), raw, raw, 1, 0, scale)
+    for t, p in enumerate((40, 9)):
+        ref, rl = causal_attention(bf16_bits_to_f64(q[t]), bf16_bits_to_f64(raw[t, :p + 1]), scale)
+        assert np.allclose(of[t], ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_end_to_end_tiny(o):
+    """The chain compress -> query -> score -> top-k -> attend on a tiny
+    case equals a direct numpy/scipy construction of the same quantities."""
+    rng = np.random.default_rng(18)
+    m, L, D, r, Hi, H, k, W = 4, 48, 32, 16, 2, 16, 5, 6
+    raw = rand_bf16(rng, (1, L, 128))
+    rawk = rand_bf16(rng, (1, L, 64))
+    z = np.full((m, 128), -np.inf, np.float32)
+    z[2] = 0
+    zk = np.full((m, 64), -np.inf, np.float32)
+    zk[2] = 0
+    comp, _ = o.compress(raw, np.array([L], np.int32), z, 0, 1 << 30)
+    kid, _ = o.compress(rawk, np.array([L], np.int32), zk, 0, 1 << 30)
+    h = rand_bf16(rng, (1, D))
+    W_dq, W_uq, W_w = rand_bf16(rng, (r, D)), rand_bf16(rng, (Hi * 64, r)), rand_bf16(rng, (Hi, D))
+    qi, wi = o.index_query(h, W_dq, W_uq, W_w)
+    p = L - 3
+    S = o.index_scores(qi, wi, [0], [p], kid, m, L // m)
+    idx, _ = o.topk(S, np.array([p], np.int32), m, k)
+    qa = rand_bf16(rng, (1, H, 128))
+    out, _ = o.sparse_attend(qa, [0], [p], comp, raw, m, idx, W, 128 ** -0.5)
+    # direct construction
+    keys = bf16_bits_to_f64(rawk[0, 2::m])                 # one-hot pooling = subsample
+    u = bf16_bits_to_f64(h) @ bf16_bits_to_f64(W_dq).T
+    qq = (u @ bf16_bits_to_f64(W_uq).T).reshape(Hi, 64)
+    ww = (bf16_bits_to_f64(h) @ bf16_bits_to_f64(W_w).T)[0]
+    V = (p + 1) // m
+    sc = (ww[:, None] * np.maximum(qq @ keys[:V].T, 0)).sum(0)
+    sel = np.lexsort((np.arange(V), -sc))[:k]
+    rows = np.concatenate([bf16_bits_to_f64(raw[0, 2::m])[sel], bf16_bits_to_f64(raw[0, p - W + 1:p + 1])])
+    ref, _ = causal_attention(bf16_bits_to_f64(qa[0]), rows, 128 ** -0.5)
+    assert np.array_equal(idx[0], sel)
+    assert np.allclose(out[0], ref, rtol=1e-12, atol=1e-12)
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

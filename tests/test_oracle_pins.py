@@ -1,0 +1,44 @@
+"""The oracle against its pins (CPU), and the pins against planted mistakes.
+
+A pin that cannot tell a wrong oracle from the right one pins nothing, so
+each planted build (oracle.c compiled with -DORACLE_PLANT=n: an off-by-one
+row, a transposed softmax, a dropped ReLU or head weight, a reversed
+tie-break, a dropped window row, a dropped softmax scale, an off-by-one
+visibility rule, truncating E4M3 rounding, HCA without its window) must fail
+at least one pin.
+"""
+import pytest
+
+import oracle as oracle_pkg
+from tests import pins
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(pin, oracle):
+    pin(oracle)
+
+
+PLANTS = {
+    1: "compress reads the wrong row (off by one)",
+    2: "pooling softmax over channels instead of positions",
+    3: "indexer ReLU dropped",
+    4: "indexer head weight dropped",
+    5: "top-k ties broken by index descending",
+    6: "window drops the query's own raw row",
+    7: "attention softmax scale dropped",
+    8: "visibility rule off by one",
+    9: "E4M3 rounding truncates",
+    10: "HCA attends without its window",
+}
+
+
+@pytest.mark.parametrize("plant", sorted(PLANTS), ids=lambda n: f"plant{n}")
+def test_pins_catch_planted_mistake(plant):
+    bad = oracle_pkg.get(plant)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(bad)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught planted mistake {plant}: {PLANTS[plant]}"
