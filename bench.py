@@ -1,0 +1,383 @@
+#!/usr/bin/env python
+"""Throughput of the CSA decode hot path at 1M-token context on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload csa_decode_1m|csa_decode_64k|csa_decode_4k|hca_decode_1m]
+                    [--kidx bf16|fp8]
+
+A step is one decode pass of the whole hot path for every sequence of the
+batch: refresh the newest compressed block, indexer query projection, score
+every visible compressed block + exact top-k, sparse attention over the
+selected blocks and the raw window.  Inputs are synthetic and seeded
+(``long_context_sparse_03_b200.workloads``); the caches stay resident in HBM.
+L2 is flushed (a 256 MiB write) before every timed step.
+
+Prints one JSON line (rank 0).  With --gpus N > 1 (under torchrun) every rank
+decodes its own batch of independent sequences (weak scaling, no
+collective on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_03_b200 import workloads as wl  # noqa: E402
+
+WORKLOADS = {"csa_decode_1m": wl.CSA_DECODE_1M, "csa_decode_64k": wl.CSA_DECODE_64K_RAGGED,
+             "csa_decode_4k": wl.CSA_DECODE_4K, "hca_decode_1m": wl.HCA_DECODE_1M}
+METRIC = "CSA decode tokens/s and achieved HBM GB/s at 1M context, 1xB200"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- ranks
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank decodes its own independent batch."""
+    return seed + 7919 * rank
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        try:
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.gpu = str(device.index)
+        self.samples = []
+        self._stop = threading.Event()
+        self._th = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._th = threading.Thread(target=self._run, daemon=True)
+        self._th.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._th:
+            self._th.join(timeout=10)
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for s in self.samples for n, v in zip(names, s[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def measured_hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------- oracle leg
+def oracle_inputs(inp, w):
+    """Host copies of the seeded inputs and the oracle's own caches
+    (untimed set-up of the CPU baseline)."""
+    import oracle
+    o = oracle.get()
+    from long_context_sparse_03_b200.workloads import bits
+    raw_kv = bits(inp.raw_kv)
+    raw_ki = bits(inp.raw_ki)
+    lens = inp.lens.cpu().numpy()
+    z_kv, z_ki = inp.z_kv.cpu().numpy(), inp.z_ki.cpu().numpy()
+    comp, _ = o.compress(raw_kv, lens, z_kv, 0, 1 << 30)
+    kid = None
+    if w.kind != "hca_decode":
+        kid, _ = o.compress(raw_ki, lens, z_ki, 0, 1 << 30)
+    return dict(o=o, raw_kv=raw_kv, raw_ki=raw_ki, lens=lens, z_kv=z_kv, z_ki=z_ki, comp=comp, kid=kid,
+                h=bits(inp.h), W_dq=bits(inp.W_dq), W_uq=bits(inp.W_uq), W_w=bits(inp.W_w), q=bits(inp.q),
+                q_seq=inp.q_seq.cpu().numpy(), q_pos=inp.q_pos.cpu().numpy())
+
+
+def oracle_step(d, w):
+    """One decode step of the oracle (the same stages as the GPU step)."""
+    o = d["o"]
+    o.compress(d["raw_kv"], d["lens"], d["z_kv"], -1, 1, out=d["comp"])
+    if w.kind == "hca_decode":
+        return o.hca_attend(d["q"], d["q_seq"], d["q_pos"], d["comp"], d["raw_kv"], w.m, w.W, 128 ** -0.5)
+    o.compress(d["raw_ki"], d["lens"], d["z_ki"], -1, 1, out=d["kid"])
+    qi, wi = o.index_query(d["h"], d["W_dq"], d["W_uq"], d["W_w"])
+    S = o.index_scores(qi, wi, d["q_seq"], d["q_pos"], d["kid"], w.m, w.max_blocks)
+    idx, _ = o.topk(S, d["q_pos"], w.m, w.k)
+    return o.sparse_attend(d["q"], d["q_seq"], d["q_pos"], d["comp"], d["raw_kv"], w.m, idx, w.W, 128 ** -0.5)
+
+
+def time_oracle(d, w, steps: int, budget_s: float = 30.0):
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(steps):
+        oracle_step(d, w)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done, dt
+
+
+# ---------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="csa_decode_1m")
+    ap.add_argument("--kidx", choices=["bf16", "fp8"], default="bf16")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="replay each step as a captured CUDA graph")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    w0 = WORKLOADS[args.workload]
+    w = wl.scaled(w0, seed=rank_seed(w0.seed, rank))
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world, dev)
+
+    from long_context_sparse_03_b200 import csa
+    from long_context_sparse_03_b200.decode import CsaDecoder, HcaDecoder
+    csa.lib()
+    inp = wl.make_inputs(w, device=str(dev))
+    stream = torch.cuda.current_stream()
+    hca = w.kind == "hca_decode"
+    fmt = csa.FMT_BF16 if args.kidx == "bf16" else csa.FMT_FP8E4M3
+    dec = HcaDecoder(inp, stream) if hca else CsaDecoder(inp, fmt, stream)
+
+    # cache build, timed on its own (bulk compression stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    dec.build_caches()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    raw_bytes = inp.raw_kv.numel() * 2 + (0 if hca else inp.raw_ki.numel() * 2)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evk = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+
+    graph = None
+    if args.graph:
+        dec.step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            dec.step()
+
+    def one(i=None):
+        if graph is not None:
+            if i is not None:
+                ev[i][0].record(stream)
+            graph.replay()
+            if i is not None:
+                ev[i][1].record(stream)
+            return
+        if i is not None:
+            ev[i][0].record(stream)
+        dec.step(evk[i] if i is not None else None)
+        if i is not None:
+            ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        one()
+    torch.cuda.synchronize()
+    barrier(dev)
+    torch.cuda.synchronize()
+    n0 = csa.launch_count()
+    with ClockSampler(dev) as clk:
+        for i in range(args.steps):
+            flush.fill_(1)
+            one(i)
+        torch.cuda.synchronize()
+    launches = csa.launch_count() - n0
+    barrier(dev)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(step_ms))
+    total_ms_max = reduce_max(total_ms, dev)
+    ms_per_step = total_ms_max / args.steps
+    tokens = reduce_sum(dec.T * args.steps, dev)
+    value = tokens / (total_ms_max / 1e3)
+    ab = dec.algorithmic_bytes()
+    step_gbs = ab["total"] / (ms_per_step / 1e3) / 1e9
+
+    # dominant kernel: the indexer scoring stream (CSA) or the dense attention (HCA)
+    peak, peak_src = measured_hbm_peak()
+    if graph is None and not hca:
+        k_ms = float(np.mean([a.elapsed_time(b) for a, b in evk]))
+        kbytes = ab["keys"]
+        kname = "index_score_kernel"
+    elif graph is None:
+        k_ms = float(np.mean([a.elapsed_time(b) for a, b in evk]))
+        kbytes = ab["total"]
+        kname = "attend_kernel+combine_kernel"
+    else:
+        k_ms, kbytes, kname = None, None, None
+    roof = None
+    if k_ms:
+        ach = kbytes / (k_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": kname, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "peak_source": peak_src, "traffic": None,
+                "algorithmic_bytes_per_launch": kbytes, "avg_launch_ms": round(k_ms, 5)}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not hca and world >= 1:
+        B = w.B
+        h_host = inp.h.cpu().pin_memory()
+        q_host = inp.q.cpu().pin_memory()
+        pos = inp.lens.long() - 1
+        bidx = torch.arange(B, device=dev)
+        kv_row = inp.raw_kv[bidx, pos].cpu().pin_memory()
+        ki_row = inp.raw_ki[bidx, pos].cpu().pin_memory()
+        out_host = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            dec.step_host(h_host, q_host, kv_row, ki_row, out_host)
+        torch.cuda.synchronize()
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(1)
+            ee[i][0].record(stream)
+            dec.step_host(h_host, q_host, kv_row, ki_row, out_host)
+            ee[i][1].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(float(sum(a.elapsed_time(b) for a, b in ee)), dev)
+        h2d = h_host.numel() * 2 + q_host.numel() * 2 + kv_row.numel() * 2 + ki_row.numel() * 2
+        e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(out_host.numel() * 2)}
+
+    # CPU baseline: the oracle on this workload's host cores (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        d = oracle_inputs(inp, w)
+        done, dt = time_oracle(d, w, steps=max(1, args.steps), budget_s=20.0)
+        cpu = {"value": round(done * dec.T / dt, 3), "unit": "tokens/s", "cores": d["o"].num_threads(),
+               "kind": "oracle",
+               "sample": f"{done} full decode step(s) of all {dec.T} sequences (double-precision C oracle, "
+                         f"OpenMP over queries), caches built untimed"}
+
+    if rank == 0:
+        rec = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if fmt == 0 else "bf16+e4m3",
+            "data": "synthetic (seeded N(0,1), weights 1/sqrt(fan_in)); caches resident in HBM",
+            "config": {"workload": w0.name, "B_per_gpu": w.B, "context": w.L, "m": w.m, "k": w.k, "W": w.W,
+                       "H": w.H, "Hi": w.Hi, "d_model": w.D, "rank": w.r,
+                       "indexer_keys": args.kidx, "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"replicas x{world} (independent batches per GPU)",
+                       "cuda_graph": bool(args.graph)},
+            "step_hbm_gbs": round(step_gbs, 1), "step_algorithmic_bytes": ab["total"],
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clk.summary(),
+            "cache_build": {"ms": round(build_ms, 3), "raw_bytes_read": raw_bytes,
+                            "gbs": round(raw_bytes / (build_ms / 1e3) / 1e9, 1)},
+        }
+        print(json.dumps(rec), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        graph = None
+        dist.destroy_process_group()
+
+
+def run_reference(args, w, rank, world, dev):
+    """The oracle arm: the CPU oracle timed on this workload's host cores."""
+    if rank != 0:
+        return
+    inp = wl.make_inputs(w, device=str(dev))
+    d = oracle_inputs(inp, w)
+    for _ in range(min(1, args.warmup)):
+        oracle_step(d, w)
+    done, dt = time_oracle(d, w, steps=args.steps, budget_s=120.0)
+    T = int(inp.T)
+    val = done * T / dt
+    rec = {"impl": "reference", "metric": METRIC, "value": round(val, 3), "unit": "tokens/s", "n_gpus": world,
+           "steps": done, "warmup": args.warmup, "ms_per_step": round(dt / done * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs)",
+           "config": {"workload": WORKLOADS[args.workload].name, "B_per_gpu": w.B, "context": w.L, "m": w.m,
+                      "k": w.k, "W": w.W, "H": w.H, "Hi": w.Hi, "d_model": w.D, "rank": w.r},
+           "cpu_baseline": {"value": round(val, 3), "unit": "tokens/s", "cores": d["o"].num_threads(),
+                            "kind": "oracle",
+                            "sample": f"{done} full decode step(s) of all {T} sequences; caches built untimed"},
+           "e2e": {"value": round(val, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(rec), flush=True)
+
+
+if __name__ == "__main__":
+    main()

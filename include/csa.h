@@ -61,6 +61,14 @@
 extern "C" {
 #endif
 
+/* Symbols of the C ABI are exported with default visibility (the library
+ * itself is built with hidden visibility for everything else). */
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
 /* Same object as cudaStream_t (CUDA defines it as struct CUstream_st*). */
 struct CUstream_st;
 typedef struct CUstream_st* csa_stream_t;
@@ -92,25 +100,25 @@ enum { CSA_DEV_BAD_INDEX = 1u, CSA_DEV_TIMEOUT = 2u };
 /* attention heads H: 16, 32, 48, ..., 128 (a multiple of 16) */
 
 /* Human-readable name of a status code (static string). */
-const char* csa_status_string(csa_status s);
+CSA_API const char* csa_status_string(csa_status s);
 
 /* Detail of the last error on the calling host thread (static per thread;
  * empty string after a successful call). */
-const char* csa_last_error(void);
+CSA_API const char* csa_last_error(void);
 
 /* Number of kernels this library has launched since it was loaded (all
  * threads).  Used to count device launches in a timed region. */
-uint64_t csa_launch_count(void);
+CSA_API uint64_t csa_launch_count(void);
 
 /* Bytes reserved at the start of every workspace for the status word. */
 #define CSA_WS_HEADER_BYTES 256
 
 /* Zero the status word of a freshly allocated workspace (async). */
-csa_status csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream);
+CSA_API csa_status csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* Synchronise `stream`, read the workspace's status word, clear it.
  * Returns CSA_OK, or CSA_ERR_DEVICE with the bits in csa_last_error(). */
-csa_status csa_status_check(void* ws, size_t ws_bytes, csa_stream_t stream);
+CSA_API csa_status csa_status_check(void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* ------------------------------------------------------------------ */
 /* 1. Compression (CSA bullet: "combining adjacent entries"; HCA bullet:  */
@@ -136,7 +144,7 @@ csa_status csa_status_check(void* ws, size_t ws_bytes, csa_stream_t stream);
  * Accumulation: fp32, one FMA per position in order i = 0..m-1; bf16 output
  * rounded to nearest even.  Blocks outside the range are not written.
  */
-csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* lens,
+CSA_API csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* lens,
                         int B, int d, int m, const float* pool_logits,
                         int blk_lo, int blk_hi,
                         void* out, int64_t out_seq_stride, int out_fmt,
@@ -149,7 +157,7 @@ csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* 
 /* ------------------------------------------------------------------ */
 
 /* Workspace for csa_index_query / csa_index_select / csa_index_topk. */
-size_t csa_index_workspace_size(int T, int r, int Hi, int k, int max_blocks);
+CSA_API size_t csa_index_workspace_size(int T, int r, int Hi, int k, int max_blocks);
 
 /*
  * Indexer query projection.  h bf16 [T][D]; W_dq bf16 [r][D]; W_uq bf16
@@ -157,7 +165,7 @@ size_t csa_index_workspace_size(int T, int r, int Hi, int k, int max_blocks);
  * (not rounded further).  u = W_dq h is kept in fp32 (workspace).
  * Constraints: D % 8 == 0, r % 8 == 0, 1 <= Hi <= 16.
  */
-csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
+CSA_API csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
                            const void* W_dq, const void* W_uq, const void* W_w,
                            float* q_out, float* w_out,
                            void* ws, size_t ws_bytes, csa_stream_t stream);
@@ -169,7 +177,7 @@ csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
  * fp32 [B][scale_seq_stride] (CSA_FMT_FP8E4M3).  Uses the same scoring
  * arithmetic as csa_index_select.
  */
-csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq,
+CSA_API csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq,
                             const int32_t* q_pos, int T, int Hi,
                             const void* kidx, int kidx_fmt, const float* kidx_scale,
                             int64_t kidx_seq_stride, int64_t scale_seq_stride,
@@ -184,7 +192,7 @@ csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq
  * exact local top-k, which later stages merge.  Equivalent to
  * csa_index_stage_score followed by csa_index_stage_merge.
  */
-csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq,
+CSA_API csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq,
                             const int32_t* q_pos, int T, int Hi,
                             const void* kidx, int kidx_fmt, const float* kidx_scale,
                             int64_t kidx_seq_stride, int64_t scale_seq_stride,
@@ -194,7 +202,7 @@ csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq
 
 /* First stage of csa_index_select: the streaming score kernel, writing the
  * per-chunk exact top-k candidates into the workspace. */
-csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* q_seq,
+CSA_API csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* q_seq,
                                  const int32_t* q_pos, int T, int Hi,
                                  const void* kidx, int kidx_fmt, const float* kidx_scale,
                                  int64_t kidx_seq_stride, int64_t scale_seq_stride,
@@ -203,12 +211,12 @@ csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* 
 
 /* Second stage: merge the candidates left in the workspace by
  * csa_index_stage_score (same T, max_blocks, k) into out_idx / out_score. */
-csa_status csa_index_stage_merge(int T, int max_blocks, int k,
+CSA_API csa_status csa_index_stage_merge(int T, int max_blocks, int k,
                                  int32_t* out_idx, float* out_score,
                                  void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* csa_index_query followed by csa_index_select. */
-csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq,
+CSA_API csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq,
                           const void* W_uq, const void* W_w,
                           const int32_t* q_seq, const int32_t* q_pos, int T, int Hi,
                           const void* kidx, int kidx_fmt, const float* kidx_scale,
@@ -224,7 +232,7 @@ csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq,
 
 /* Workspace for csa_sparse_attend (max_rows = k + W) and hca_attend
  * (max_rows = max_blocks + W). */
-size_t csa_attend_workspace_size(int T, int H, int max_rows);
+CSA_API size_t csa_attend_workspace_size(int T, int H, int max_rows);
 
 /*
  * q bf16 [T][H][128]; comp bf16 compressed latent rows [B][.][128] (row j at
@@ -236,7 +244,7 @@ size_t csa_attend_workspace_size(int T, int H, int max_rows);
  * fp32 logits, softmax and accumulation; split-K over fixed 128-row
  * splits merged in a fixed order.
  */
-csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
+CSA_API csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
                              int T, int H, const void* comp, int64_t comp_seq_stride,
                              const void* raw, int64_t raw_seq_stride, int m,
                              const int32_t* idx, int k, int W, float scale,
@@ -245,7 +253,7 @@ csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t*
 
 /* HCA: as csa_sparse_attend with the attended compressed rows being every
  * visible block j < min(V(t), max_blocks) (m = m'). */
-csa_status hca_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
+CSA_API csa_status hca_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
                       int T, int H, const void* comp, int64_t comp_seq_stride,
                       const void* raw, int64_t raw_seq_stride, int m, int max_blocks,
                       int W, float scale, void* out, float* lse,

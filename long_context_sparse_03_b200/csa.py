@@ -1,0 +1,233 @@
+"""ctypes binding of libcsa.so (the C ABI in include/csa.h).
+
+Argument marshalling only: every function here passes torch device tensors'
+pointers and sizes to the C call of the same name and raises ``CsaError``
+on a non-OK status.  No arithmetic of the method runs in Python, and there
+is no fallback: without the built library, loading raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from pathlib import Path
+
+import torch
+
+_HERE = Path(__file__).resolve().parent
+LIB_PATH = _HERE / "libcsa.so"
+HEADER = _HERE.parent / "include" / "csa.h"
+
+FMT_BF16 = 0
+FMT_FP8E4M3 = 1
+WS_HEADER_BYTES = 256
+
+STATUS = {0: "CSA_OK", 1: "CSA_ERR_NULL", 2: "CSA_ERR_SHAPE", 3: "CSA_ERR_UNSUPPORTED",
+          4: "CSA_ERR_WORKSPACE", 5: "CSA_ERR_CUDA", 6: "CSA_ERR_TIMEOUT", 7: "CSA_ERR_DEVICE",
+          8: "CSA_ERR_ALIGN"}
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, func: str, detail: str):
+        super().__init__(f"{func}: {STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+_P, _I, _L, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "csa_status_string": (ctypes.c_char_p, [_I]),
+    "csa_last_error": (ctypes.c_char_p, []),
+    "csa_launch_count": (ctypes.c_uint64, []),
+    "csa_workspace_init": (_I, [_P, _S, _P]),
+    "csa_status_check": (_I, [_P, _S, _P]),
+    "csa_compress": (_I, [_P, _L, _P, _I, _I, _I, _P, _I, _I, _P, _L, _I, _P, _L, _P]),
+    "csa_index_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "csa_index_query": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "csa_index_scores": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _P, _P]),
+    "csa_index_select": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _I, _P, _P, _P, _S, _P]),
+    "csa_index_stage_score": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _I, _P, _S, _P]),
+    "csa_index_stage_merge": (_I, [_I, _I, _I, _P, _P, _P, _S, _P]),
+    "csa_index_topk": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _I, _P, _P,
+                            _P, _S, _P]),
+    "csa_attend_workspace_size": (_S, [_I, _I, _I]),
+    "csa_sparse_attend": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _P, _I, _I, _F, _P, _P, _P, _S, _P]),
+    "hca_attend": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _I, _I, _F, _P, _P, _P, _S, _P]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libcsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m long_context_sparse_03_b200.build`")
+        L = ctypes.CDLL(str(LIB_PATH))
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/csa.h."""
+    text = HEADER.read_text()
+    return sorted(set(re.findall(r"CSA_API\s+[\w\s\*]+?\b((?:csa|hca)_\w+)\s*\(", text)))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(stream)
+
+
+def _check(status: int, func: str):
+    if status != 0:
+        raise CsaError(status, func, lib().csa_last_error().decode())
+
+
+def launch_count() -> int:
+    return int(lib().csa_launch_count())
+
+
+def _seq_stride(t: torch.Tensor) -> int:
+    return int(t.stride(0)) if t.dim() >= 3 else 0
+
+
+# ---------------------------------------------------------------- workspace
+class Workspace:
+    """A device byte buffer handed to the library as scratch."""
+
+    def __init__(self, nbytes: int, device="cuda", stream=None):
+        self.nbytes = int(max(nbytes, WS_HEADER_BYTES))
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        _check(lib().csa_workspace_init(_ptr(self.buf), self.nbytes, _stream(stream)), "csa_workspace_init")
+
+    def ptr(self):
+        return _ptr(self.buf)
+
+    def check(self, stream=None):
+        """Raise CsaError if a kernel flagged an anomaly (syncs the stream)."""
+        _check(lib().csa_status_check(self.ptr(), self.nbytes, _stream(stream)), "csa_status_check")
+
+
+def csa_index_workspace_size(T, r, Hi, k, max_blocks) -> int:
+    return int(lib().csa_index_workspace_size(T, r, Hi, k, max_blocks))
+
+
+def csa_attend_workspace_size(T, H, max_rows) -> int:
+    return int(lib().csa_attend_workspace_size(T, H, max_rows))
+
+
+# ---------------------------------------------------------------- calls
+def csa_compress(raw, lens, pool_logits, m, blk_lo, blk_hi, out, out_fmt=FMT_BF16, out_scale=None,
+                 stream=None):
+    """raw [B][L][d] bf16, lens int32 [B], pool_logits fp32 [m][d]; writes out (and out_scale)."""
+    B, _, d = raw.shape
+    st = lib().csa_compress(_ptr(raw), raw.stride(0), _ptr(lens), B, d, m, _ptr(pool_logits), blk_lo, blk_hi,
+                            _ptr(out), out.stride(0), out_fmt, _ptr(out_scale),
+                            0 if out_scale is None else out_scale.stride(0), _stream(stream))
+    _check(st, "csa_compress")
+    return out, out_scale
+
+
+def csa_index_query(h, W_dq, W_uq, W_w, q_out, w_out, ws: Workspace, stream=None):
+    T, D = h.shape
+    r = W_dq.shape[0]
+    Hi = W_w.shape[0]
+    st = lib().csa_index_query(_ptr(h), T, D, r, Hi, _ptr(W_dq), _ptr(W_uq), _ptr(W_w), _ptr(q_out),
+                               _ptr(w_out), ws.ptr(), ws.nbytes, _stream(stream))
+    _check(st, "csa_index_query")
+    return q_out, w_out
+
+
+def _kidx_args(kidx, kidx_scale):
+    fmt = FMT_BF16 if kidx.dtype == torch.bfloat16 else FMT_FP8E4M3
+    return fmt, kidx.stride(0), (0 if kidx_scale is None else kidx_scale.stride(0))
+
+
+def csa_index_scores(q, w, q_seq, q_pos, kidx, m, max_blocks, scores, kidx_scale=None, stream=None):
+    T, Hi, _ = q.shape
+    fmt, ks, ss = _kidx_args(kidx, kidx_scale)
+    st = lib().csa_index_scores(_ptr(q), _ptr(w), _ptr(q_seq), _ptr(q_pos), T, Hi, _ptr(kidx), fmt,
+                                _ptr(kidx_scale), ks, ss, m, max_blocks, _ptr(scores), _stream(stream))
+    _check(st, "csa_index_scores")
+    return scores
+
+
+def csa_index_select(q, w, q_seq, q_pos, kidx, m, max_blocks, k, out_idx, out_score, ws: Workspace,
+                     kidx_scale=None, stream=None):
+    T, Hi, _ = q.shape
+    fmt, ks, ss = _kidx_args(kidx, kidx_scale)
+    st = lib().csa_index_select(_ptr(q), _ptr(w), _ptr(q_seq), _ptr(q_pos), T, Hi, _ptr(kidx), fmt,
+                                _ptr(kidx_scale), ks, ss, m, max_blocks, k, _ptr(out_idx), _ptr(out_score),
+                                ws.ptr(), ws.nbytes, _stream(stream))
+    _check(st, "csa_index_select")
+    return out_idx, out_score
+
+
+def csa_index_stage_score(q, w, q_seq, q_pos, kidx, m, max_blocks, k, ws: Workspace, kidx_scale=None,
+                          stream=None):
+    T, Hi, _ = q.shape
+    fmt, ks, ss = _kidx_args(kidx, kidx_scale)
+    st = lib().csa_index_stage_score(_ptr(q), _ptr(w), _ptr(q_seq), _ptr(q_pos), T, Hi, _ptr(kidx), fmt,
+                                     _ptr(kidx_scale), ks, ss, m, max_blocks, k, ws.ptr(), ws.nbytes,
+                                     _stream(stream))
+    _check(st, "csa_index_stage_score")
+
+
+def csa_index_stage_merge(T, max_blocks, k, out_idx, out_score, ws: Workspace, stream=None):
+    st = lib().csa_index_stage_merge(T, max_blocks, k, _ptr(out_idx), _ptr(out_score), ws.ptr(), ws.nbytes,
+                                     _stream(stream))
+    _check(st, "csa_index_stage_merge")
+
+
+def csa_index_topk(h, W_dq, W_uq, W_w, q_seq, q_pos, kidx, m, max_blocks, k, out_idx, out_score,
+                   ws: Workspace, kidx_scale=None, stream=None):
+    T, D = h.shape
+    r = W_dq.shape[0]
+    Hi = W_w.shape[0]
+    fmt, ks, ss = _kidx_args(kidx, kidx_scale)
+    st = lib().csa_index_topk(_ptr(h), D, r, _ptr(W_dq), _ptr(W_uq), _ptr(W_w), _ptr(q_seq), _ptr(q_pos), T, Hi,
+                              _ptr(kidx), fmt, _ptr(kidx_scale), ks, ss, m, max_blocks, k, _ptr(out_idx),
+                              _ptr(out_score), ws.ptr(), ws.nbytes, _stream(stream))
+    _check(st, "csa_index_topk")
+    return out_idx, out_score
+
+
+def csa_sparse_attend(q, q_seq, q_pos, comp, raw, m, idx, W, scale, out, lse, ws: Workspace, stream=None):
+    T, H, _ = q.shape
+    k = idx.shape[1]
+    st = lib().csa_sparse_attend(_ptr(q), _ptr(q_seq), _ptr(q_pos), T, H, _ptr(comp), comp.stride(0), _ptr(raw),
+                                 raw.stride(0), m, _ptr(idx), k, W, float(scale), _ptr(out), _ptr(lse), ws.ptr(),
+                                 ws.nbytes, _stream(stream))
+    _check(st, "csa_sparse_attend")
+    return out, lse
+
+
+def hca_attend(q, q_seq, q_pos, comp, raw, m, max_blocks, W, scale, out, lse, ws: Workspace, stream=None):
+    T, H, _ = q.shape
+    st = lib().hca_attend(_ptr(q), _ptr(q_seq), _ptr(q_pos), T, H, _ptr(comp), comp.stride(0), _ptr(raw),
+                          raw.stride(0), m, max_blocks, W, float(scale), _ptr(out), _ptr(lse), ws.ptr(), ws.nbytes,
+                          _stream(stream))
+    _check(st, "hca_attend")
+    return out, lse
+
+
+def softmax_scale(d: int = 128) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,107 @@
+// common.cuh -- device helpers shared by the libcsa kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+typedef __nv_bfloat16 bf16;
+
+// Device status bits, mirrored from include/csa.h.
+constexpr unsigned kDevBadIndex = 1u;
+constexpr unsigned kDevTimeout = 2u;
+
+constexpr int kWsHeader = 256;
+
+__device__ __forceinline__ void flag_status(unsigned* status, unsigned bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// ---------------------------------------------------------------- ordering
+// fp32 score -> uint32 whose unsigned order is the float order (+0 and -0
+// map to the same key, so they tie and the block index decides).
+__device__ __forceinline__ uint32_t score_key(float s) {
+    uint32_t u = __float_as_uint(s);
+    if ((u & 0x7FFFFFFFu) == 0u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+    return __uint_as_float(u);
+}
+// (score desc, index asc) as one descending uint64; 0 is the empty slot
+// (it decodes to index -1 and is below every real entry).
+__device__ __forceinline__ uint64_t make_cand(float s, int j) {
+    return ((uint64_t)score_key(s) << 32) | (uint32_t)(~(uint32_t)j);
+}
+__device__ __forceinline__ int cand_index(uint64_t c) { return (int)(~(uint32_t)(c & 0xFFFFFFFFu)); }
+__device__ __forceinline__ float cand_score(uint64_t c) { return key_score((uint32_t)(c >> 32)); }
+
+// ---------------------------------------------------------------- MMA
+// mma.sync m16n8k16, fp32 accumulate.  Fragment ownership for lane
+// (g = lane / 4, tq = lane % 4):
+//   A: r0 = (row g, k 2tq..2tq+1)   r1 = (row g+8, k 2tq..2tq+1)
+//      r2 = (row g, k 2tq+8..+9)    r3 = (row g+8, k 2tq+8..+9)
+//   B: r0 = (k 2tq..2tq+1, col g)   r1 = (k 2tq+8..+9, col g)
+//   C: c0,c1 = (row g, cols 2tq, 2tq+1)  c2,c3 = (row g+8, same cols)
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low half)
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t* r, const void* smem_row) {
+    uint32_t a = (uint32_t)__cvta_generic_to_shared(smem_row);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t* r, const void* smem_row) {
+    uint32_t a = (uint32_t)__cvta_generic_to_shared(smem_row);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(a));
+}
+
+// ---------------------------------------------------------------- memory
+// 16-byte global load that bypasses L1 (each key is read once).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// cp.async 16 B global -> shared; src_bytes = 0 zero-fills the destination.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, int src_bytes) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+}  // namespace csa

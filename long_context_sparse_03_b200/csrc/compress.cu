@@ -1,0 +1,141 @@
+// compress.cu -- KV / indexer-key compression by m adjacent rows.
+//
+// DeepSeek-V4 summary (b-lab.team), "Core Methodological Innovations" 1:
+// CSA compresses the KV cache by m "by combining adjacent entries"; HCA does
+// the same with m' >> m.  Reading taken: a fixed per-position, per-channel
+// weighted sum whose weights are a softmax over the m positions.
+//
+// Layout: one thread owns one 16-byte chunk (8 channels) of one output row,
+// so a warp reads whole 256-byte (d = 128) or 128-byte (d = 64) raw rows with
+// coalesced 128-bit loads, streaming m rows per output row.  The pooling
+// weights are computed once per CTA into shared memory.
+#include "common.cuh"
+
+namespace csa {
+
+template <int D, int FMT>
+__global__ void __launch_bounds__(256) compress_kernel(
+    const bf16* __restrict__ raw, int64_t raw_stride, const int* __restrict__ lens, int m,
+    const float* __restrict__ logits, int blk_lo, int blk_hi, void* __restrict__ out,
+    int64_t out_stride, float* __restrict__ out_scale, int64_t scale_stride) {
+    constexpr int TPR = D / 8;            // threads per output row
+    constexpr int RPC = 256 / TPR;        // output rows per CTA
+    extern __shared__ float a_sh[];       // [m][D] pooling weights
+
+    for (int c = threadIdx.x; c < D; c += blockDim.x) {
+        float mx = -INFINITY;
+        for (int i = 0; i < m; ++i) mx = fmaxf(mx, logits[i * D + c]);
+        float sum = 0.f;
+        for (int i = 0; i < m; ++i) sum += expf(logits[i * D + c] - mx);
+        for (int i = 0; i < m; ++i) a_sh[i * D + c] = expf(logits[i * D + c] - mx) / sum;
+    }
+    __syncthreads();
+
+    const int b = blockIdx.y;
+    const int nblk = lens[b] / m;
+    int lo, hi;
+    if (blk_lo >= 0) {
+        lo = blk_lo;
+        hi = min(blk_hi, nblk);
+    } else {
+        lo = max(0, nblk - blk_hi);
+        hi = nblk;
+    }
+    const int j = lo + blockIdx.x * RPC + threadIdx.x / TPR;
+    const int chunk = threadIdx.x % TPR;
+    if (j >= hi) return;
+
+    const bf16* src = raw + (int64_t)b * raw_stride + (int64_t)j * m * D + chunk * 8;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < m; ++i) {
+        uint4 v = ldg_stream(src + (int64_t)i * D);
+        const float4 w0 = *reinterpret_cast<const float4*>(&a_sh[i * D + chunk * 8]);
+        const float4 w1 = *reinterpret_cast<const float4*>(&a_sh[i * D + chunk * 8 + 4]);
+        const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&v);
+        float2 x0 = __bfloat1622float2(x[0]), x1 = __bfloat1622float2(x[1]);
+        float2 x2 = __bfloat1622float2(x[2]), x3 = __bfloat1622float2(x[3]);
+        acc[0] = fmaf(w0.x, x0.x, acc[0]);
+        acc[1] = fmaf(w0.y, x0.y, acc[1]);
+        acc[2] = fmaf(w0.z, x1.x, acc[2]);
+        acc[3] = fmaf(w0.w, x1.y, acc[3]);
+        acc[4] = fmaf(w1.x, x2.x, acc[4]);
+        acc[5] = fmaf(w1.y, x2.y, acc[5]);
+        acc[6] = fmaf(w1.z, x3.x, acc[6]);
+        acc[7] = fmaf(w1.w, x3.y, acc[7]);
+    }
+    // bf16 row (round to nearest even)
+    uint4 ob;
+    uint32_t* obw = reinterpret_cast<uint32_t*>(&ob);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) obw[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
+
+    if (FMT == 0) {
+        bf16* dst = reinterpret_cast<bf16*>(out) + (int64_t)b * out_stride + (int64_t)j * D + chunk * 8;
+        *reinterpret_cast<uint4*>(dst) = ob;
+    } else {
+        // E4M3 row with one fp32 scale: s = amax/448 of the bf16 row.
+        float xv[8];
+        const __nv_bfloat162* xb = reinterpret_cast<const __nv_bfloat162*>(&ob);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(xb[e]);
+            xv[2 * e] = f.x;
+            xv[2 * e + 1] = f.y;
+            amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+#pragma unroll
+        for (int off = 1; off < TPR; off <<= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float s = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        uint2 codes;
+        uint16_t* cw = reinterpret_cast<uint16_t*>(&codes);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 pr = make_float2(__fdiv_rn(xv[2 * e], s), __fdiv_rn(xv[2 * e + 1], s));
+            cw[e] = __nv_cvt_float2_to_fp8x2(pr, __NV_SATFINITE, __NV_E4M3);
+        }
+        uint8_t* dst = reinterpret_cast<uint8_t*>(out) + (int64_t)b * out_stride + (int64_t)j * D + chunk * 8;
+        *reinterpret_cast<uint2*>(dst) = codes;
+        if (chunk == 0) out_scale[(int64_t)b * scale_stride + j] = s;
+    }
+}
+
+// Launch: grid.x covers the requested block range, grid.y the sequences.
+cudaError_t launch_compress(const void* raw, int64_t raw_stride, const int* lens, int B, int d, int m,
+                            const float* logits, int blk_lo, int blk_hi, void* out,
+                            int64_t out_stride, int out_fmt, float* out_scale, int64_t scale_stride,
+                            cudaStream_t stream) {
+    const int span = blk_lo >= 0 ? (blk_hi - blk_lo) : blk_hi;
+    if (span <= 0 || B <= 0) return cudaSuccess;
+    const int rpc = 256 / (d / 8);
+    dim3 grid((span + rpc - 1) / rpc, B);
+    size_t smem = sizeof(float) * (size_t)m * d;
+    const bf16* r = reinterpret_cast<const bf16*>(raw);
+    cudaError_t e = cudaSuccess;
+    if (d == 128) {
+        auto k = compress_kernel<128, 0>;
+        if (smem > 48 * 1024) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 256, smem, stream>>>(r, raw_stride, lens, m, logits, blk_lo, blk_hi, out, out_stride,
+                                       out_scale, scale_stride);
+    } else if (out_fmt == 0) {
+        auto k = compress_kernel<64, 0>;
+        if (smem > 48 * 1024) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 256, smem, stream>>>(r, raw_stride, lens, m, logits, blk_lo, blk_hi, out, out_stride,
+                                       out_scale, scale_stride);
+    } else {
+        auto k = compress_kernel<64, 1>;
+        if (smem > 48 * 1024) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        k<<<grid, 256, smem, stream>>>(r, raw_stride, lens, m, logits, blk_lo, blk_hi, out, out_stride,
+                                       out_scale, scale_stride);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -1,0 +1,159 @@
+"""One CSA or HCA decode step over resident caches, through the C ABI.
+
+``CsaDecoder`` owns the device caches of a batch of sequences (raw latent
+rows, raw indexer keys, their compressed forms) and runs the hot path of
+one decode step: refresh the newest compressed block, project the indexer
+query, score and select the top-k blocks, attend over them plus the
+window.  ``HcaDecoder`` is the heavily-compressed variant (dense attention
+over every compressed row plus the window, no indexer).  Every step is a
+sequence of libcsa calls on one stream; nothing here computes.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import csa
+from .workloads import Inputs
+
+
+class CsaDecoder:
+    def __init__(self, inp: Inputs, kidx_fmt: int = csa.FMT_BF16, stream: torch.cuda.Stream | None = None):
+        w = inp.w
+        self.inp, self.w, self.fmt = inp, w, kidx_fmt
+        self.stream = stream or torch.cuda.current_stream()
+        dev = inp.raw_kv.device
+        self.T = inp.T
+        self.N = w.max_blocks
+        self.scale = csa.softmax_scale(128)
+        self.comp = torch.empty((w.B, self.N, 128), dtype=torch.bfloat16, device=dev)
+        if kidx_fmt == csa.FMT_BF16:
+            self.kidx = torch.empty((w.B, self.N, 64), dtype=torch.bfloat16, device=dev)
+            self.kscale = None
+        else:
+            self.kidx = torch.empty((w.B, self.N, 64), dtype=torch.uint8, device=dev)
+            self.kscale = torch.empty((w.B, self.N), dtype=torch.float32, device=dev)
+        self.q_idx = torch.empty((self.T, w.Hi, 64), dtype=torch.float32, device=dev)
+        self.w_idx = torch.empty((self.T, w.Hi), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((self.T, w.k), dtype=torch.int32, device=dev)
+        self.idx_score = torch.empty((self.T, w.k), dtype=torch.float32, device=dev)
+        self.out = torch.empty((self.T, w.H, 128), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.T, w.H), dtype=torch.float32, device=dev)
+        self.ws_idx = csa.Workspace(csa.csa_index_workspace_size(self.T, w.r, w.Hi, w.k, self.N), dev, self.stream)
+        self.ws_att = csa.Workspace(csa.csa_attend_workspace_size(self.T, w.H, w.k + w.W), dev, self.stream)
+
+    # -- cache build (bulk compression of every complete block) ---------
+    def build_caches(self):
+        i, w = self.inp, self.w
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, 0, self.N, self.comp, stream=self.stream)
+        csa.csa_compress(i.raw_ki, i.lens, i.z_ki, w.m, 0, self.N, self.kidx, self.fmt, self.kscale,
+                         stream=self.stream)
+
+    # -- the step ---------------------------------------------------------
+    def refresh(self):
+        """Recompress the newest complete block of each sequence."""
+        i, w = self.inp, self.w
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, -1, 1, self.comp, stream=self.stream)
+        csa.csa_compress(i.raw_ki, i.lens, i.z_ki, w.m, -1, 1, self.kidx, self.fmt, self.kscale, stream=self.stream)
+
+    def query(self):
+        i = self.inp
+        csa.csa_index_query(i.h, i.W_dq, i.W_uq, i.W_w, self.q_idx, self.w_idx, self.ws_idx, stream=self.stream)
+
+    def score(self):
+        i, w = self.inp, self.w
+        csa.csa_index_stage_score(self.q_idx, self.w_idx, i.q_seq, i.q_pos, self.kidx, w.m, self.N, w.k, self.ws_sel,
+                                  kidx_scale=self.kscale, stream=self.stream)
+
+    def merge(self):
+        csa.csa_index_stage_merge(self.T, self.N, self.w.k, self.idx, self.idx_score, self.ws_sel, stream=self.stream)
+
+    def attend(self):
+        i, w = self.inp, self.w
+        csa.csa_sparse_attend(i.q, i.q_seq, i.q_pos, self.comp, i.raw_kv, w.m, self.idx, w.W, self.scale, self.out,
+                              self.lse, self.ws_att, stream=self.stream)
+
+    @property
+    def ws_sel(self) -> csa.Workspace:
+        # the stage calls lay their candidates out from the workspace header
+        return self.ws_idx
+
+    def step(self, ev_score: tuple | None = None):
+        """One decode step on device-resident inputs.  ev_score: optional
+        (start, end) CUDA events recorded around the scoring kernel."""
+        self.refresh()
+        self.query()
+        if ev_score:
+            ev_score[0].record(self.stream)
+        self.score()
+        if ev_score:
+            ev_score[1].record(self.stream)
+        self.merge()
+        self.attend()
+        return self.out
+
+    def step_host(self, h_host, q_host, kv_row_host, ki_row_host, out_host):
+        """The same step from pinned host buffers: copy this step's inputs
+        (hidden states, attention queries, the new token's raw rows) to the
+        device, run the step, copy the attention output back."""
+        i, s = self.inp, self.stream
+        with torch.cuda.stream(s):
+            i.h.copy_(h_host, non_blocking=True)
+            i.q.copy_(q_host, non_blocking=True)
+            pos = i.lens.long() - 1
+            bidx = torch.arange(self.w.B, device=i.raw_kv.device)
+            i.raw_kv[bidx, pos] = kv_row_host.to(i.raw_kv.device, non_blocking=True)
+            i.raw_ki[bidx, pos] = ki_row_host.to(i.raw_ki.device, non_blocking=True)
+        self.step()
+        with torch.cuda.stream(s):
+            out_host.copy_(self.out, non_blocking=True)
+        return out_host
+
+    def algorithmic_bytes(self) -> dict:
+        """Bytes the step must move: indexer keys of every visible block,
+        the gathered compressed rows and the window rows."""
+        w = self.w
+        key_b = 128 if self.fmt == csa.FMT_BF16 else 64 + 4
+        vis = ((self.inp.lens.long()) // w.m).clamp(max=self.N)
+        keys = int(vis.sum().item()) * key_b
+        gathered = int(vis.clamp(max=w.k).sum().item()) * 256
+        window = int(self.inp.lens.long().clamp(max=w.W).sum().item()) * 256
+        return {"keys": keys, "gathered": gathered, "window": window, "total": keys + gathered + window}
+
+
+class HcaDecoder:
+    """HCA decode: dense attention over all compressed rows (pooled by m')."""
+
+    def __init__(self, inp: Inputs, stream: torch.cuda.Stream | None = None):
+        w = inp.w
+        self.inp, self.w = inp, w
+        self.stream = stream or torch.cuda.current_stream()
+        dev = inp.raw_kv.device
+        self.T = inp.T
+        self.N = w.max_blocks
+        self.scale = csa.softmax_scale(128)
+        self.comp = torch.empty((w.B, self.N, 128), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((self.T, w.H, 128), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.T, w.H), dtype=torch.float32, device=dev)
+        self.ws_att = csa.Workspace(csa.csa_attend_workspace_size(self.T, w.H, self.N + w.W), dev, self.stream)
+
+    def build_caches(self):
+        i, w = self.inp, self.w
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, 0, self.N, self.comp, stream=self.stream)
+
+    def step(self, ev_attend: tuple | None = None):
+        i, w = self.inp, self.w
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, -1, 1, self.comp, stream=self.stream)
+        if ev_attend:
+            ev_attend[0].record(self.stream)
+        csa.hca_attend(i.q, i.q_seq, i.q_pos, self.comp, i.raw_kv, w.m, self.N, w.W, self.scale, self.out, self.lse,
+                       self.ws_att, stream=self.stream)
+        if ev_attend:
+            ev_attend[1].record(self.stream)
+        return self.out
+
+    def algorithmic_bytes(self) -> dict:
+        w = self.w
+        vis = (self.inp.lens.long() // w.m).clamp(max=self.N)
+        rows = int(vis.sum().item()) * 256
+        window = int(self.inp.lens.long().clamp(max=w.W).sum().item()) * 256
+        return {"compressed": rows, "window": window, "total": rows + window}

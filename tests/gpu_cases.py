@@ -1,0 +1,121 @@
+"""Shared helpers of the GPU parity tests: host<->device marshalling and the
+tolerances the CUDA path is held to against the oracle.
+
+Tolerances (each derived from the arithmetic of the kernel it judges):
+  compress   bf16 rows within 1 bf16 ulp of the oracle's, plus the error
+             bound of an fp32 chain of m fused multiply-adds, m 2^-24 sum_i
+             |a_i x_i| (it matters only when the sum cancels); bit-exact where
+             the pooling is exact (one-hot weights, m = 1).
+  E4M3 rows  bit-exact codes and scales where the bf16 row is exact; else
+             codes within one step and scales within 2^-7 relative.
+  query      |dq| <= 1e-5 * max|q| per row (fp32 dot products of <= 4096
+             bf16 products).
+  scores     |dS_j| <= 1e-3 |S_j| + 2e-5 A_j, A_j = sum_h |w_h| sum_c |q_hc k_jc|:
+             the hi+lo split keeps q to 2^-17 relative and the fp32 MMA sums 64
+             products, so the error of a head's dot is ~1e-5 of its absolute
+             sum; the 1e-3 relative part is the stated score tolerance.
+  top-k      the index sets equal the oracle's except for blocks whose oracle
+             score lies within the score tolerance of the oracle's k-th score;
+             the GPU list is valid (sorted, distinct, visible, -1 padded).
+  attention  max |d| <= 1e-2 max |ref| per call (bf16 output of fp32 softmax
+             and accumulation); lse within 1e-3 + 1e-4 |lse|.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from tests.pins import bf16_bits_to_f64
+
+
+def dev_bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def dev_i32(a) -> torch.Tensor:
+    return torch.as_tensor(np.asarray(a, np.int32)).cuda()
+
+
+# ---------------------------------------------------------------- checks
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |v| (8 significant bits)."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def check_compress_bf16(gpu_bits: np.ndarray, ref_bits: np.ndarray, exact: bool = False, absum=None, m: int = 1) -> int:
+    """absum: sum_i |a_i x_i| per element (the scale of the fp32 rounding)."""
+    g = gpu_bits.astype(np.int32)
+    r = ref_bits.astype(np.int32)
+    if exact:
+        assert np.array_equal(g, r), f"{np.count_nonzero(g != r)} of {g.size} differ"
+        return 0
+    gv, rv = bf16_bits_to_f64(gpu_bits), bf16_bits_to_f64(ref_bits)
+    # one ulp: adjacent bit patterns of the same sign (or +-0 / smallest)
+    same_sign = np.sign(gv) == np.sign(rv)
+    ulp1 = (np.abs(g - r) <= 1) & (same_sign | (np.abs(gv) < 1e-30) | (np.abs(rv) < 1e-30))
+    if absum is not None:
+        lim = bf16_ulp(rv) + m * 2.0 ** -24 * absum
+        ulp1 |= np.abs(gv - rv) <= lim
+    bad = ~ulp1
+    assert not bad.any(), f"{np.count_nonzero(bad)} elements beyond 1 bf16 ulp, e.g. {np.argwhere(bad)[:3]}"
+    return int(np.count_nonzero(g != r))
+
+
+def score_scale(q: np.ndarray, w: np.ndarray, keys: np.ndarray) -> np.ndarray:
+    """A_j = sum_h |w_h| sum_c |q_hc k_jc| for one query (keys [N][64] float64)."""
+    return np.abs(keys) @ (np.abs(q).T @ np.abs(w))
+
+
+def check_scores(gpu: np.ndarray, ref: np.ndarray, A: np.ndarray):
+    vis = ~np.isnan(ref)
+    assert np.array_equal(vis, ~np.isnan(gpu)), "visibility (NaN pattern) differs"
+    d = np.abs(gpu[vis].astype(np.float64) - ref[vis])
+    tol = 1e-3 * np.abs(ref[vis]) + 2e-5 * A[vis]
+    bad = d > tol
+    assert not bad.any(), f"{np.count_nonzero(bad)} scores off, worst ratio {np.max(d / np.maximum(tol, 1e-300)):.3g}"
+    return float(np.max(d / np.maximum(tol, 1e-300))) if d.size else 0.0
+
+
+def check_topk(gidx: np.ndarray, gscore, S: np.ndarray, A: np.ndarray, V: int, k: int):
+    """One query: GPU top-k list against the oracle scores S[0..V)."""
+    n = min(k, V)
+    assert (gidx[n:] == -1).all(), "padding"
+    sel = gidx[:n]
+    assert ((sel >= 0) & (sel < V)).all(), "index outside the visible blocks"
+    assert len(np.unique(sel)) == n, "duplicate index"
+    if gscore is not None:
+        gs = gscore[:n].astype(np.float64)
+        # sorted by GPU score desc, ties by index asc
+        for i in range(n - 1):
+            assert gs[i] > gs[i + 1] or (gs[i] == gs[i + 1] and sel[i] < sel[i + 1]), f"order at {i}"
+        assert np.isnan(gscore[n:]).all()
+        tol = 1e-3 * np.abs(S[sel]) + 2e-5 * A[sel]
+        assert (np.abs(gs - S[sel]) <= tol).all(), "returned scores"
+    if n == V:
+        return 0
+    order = np.lexsort((np.arange(V), -S[:V]))
+    ref = order[:n]
+    kth = S[ref[-1]]
+    diff = np.setxor1d(sel, ref)
+    if diff.size:
+        band = 1e-3 * np.abs(kth) + 2e-5 * np.maximum(A[diff], A[ref[-1]])
+        gap = np.abs(S[diff] - kth)
+        assert (gap <= band).all(), f"{diff.size} indices differ outside the tie band: gap {gap.max():.3g}"
+    return int(diff.size // 2)
+
+
+def check_attention(out: np.ndarray, lse, ref_out: np.ndarray, ref_lse):
+    d = np.abs(out.astype(np.float64) - ref_out)
+    lim = 1e-2 * np.abs(ref_out).max()
+    assert d.max() <= lim, f"max|d| {d.max():.3g} > {lim:.3g}"
+    if lse is not None:
+        fin = np.isfinite(ref_lse)
+        assert np.array_equal(fin, np.isfinite(lse)), "empty-set pattern of lse"
+        dl = np.abs(lse[fin] - ref_lse[fin])
+        assert (dl <= 1e-3 + 1e-4 * np.abs(ref_lse[fin])).all(), f"lse off by {dl.max():.3g}"
+    return float(d.max() / max(np.abs(ref_out).max(), 1e-30))

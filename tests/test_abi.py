@@ -1,0 +1,99 @@
+"""The C ABI on the host (no GPU needed): the library loads, exports every
+function include/csa.h declares, and rejects bad arguments before any
+launch with the documented status codes."""
+import ctypes
+
+import pytest
+
+from long_context_sparse_03_b200 import build as csa_build
+from long_context_sparse_03_b200 import csa
+
+NULL = None
+
+
+@pytest.fixture(scope="module")
+def L():
+    csa_build.build()
+    return csa.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = csa.header_functions()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(L, n), n
+    # and nothing else with the C prefixes leaks out as a public symbol
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", str(csa.LIB_PATH)], capture_output=True, text=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln})
+    assert exported == names
+
+
+def test_status_strings(L):
+    for code, name in csa.STATUS.items():
+        assert L.csa_status_string(code).decode() == name
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_compress_validation(L):
+    s = L.csa_compress
+    assert s(NULL, 0, NULL, 1, 128, 4, NULL, 0, 4, NULL, 0, 0, NULL, 0, NULL) == 1       # NULL
+    assert s(_fake(), 0, _fake(), 1, 96, 4, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 3   # d
+    assert s(_fake(), 0, _fake(), 1, 128, 0, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 3  # m
+    assert s(_fake(), 0, _fake(), 1, 128, 300, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 3
+    assert s(_fake(), 0, _fake(), 1, 128, 4, _fake(), 0, 4, _fake(), 0, 1, NULL, 0, NULL) == 3  # fp8 d=128
+    assert s(_fake(), 0, _fake(), 1, 64, 4, _fake(), 0, 4, _fake(), 0, 1, NULL, 0, NULL) == 1   # no scale
+    assert s(_fake(), 0, _fake(), 1, 128, 4, _fake(), 5, 4, _fake(), 0, 0, NULL, 0, NULL) == 2  # range
+    assert s(_fake(), 0, _fake(), 1, 128, 4, _fake(), -2, 4, _fake(), 0, 0, NULL, 0, NULL) == 2
+    assert s(_fake(0x10004), 0, _fake(), 1, 128, 4, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 8
+    assert s(_fake(), 12, _fake(), 1, 128, 4, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 8
+    # empty work is a no-op success, even with NULL pointers
+    assert s(NULL, 0, NULL, 0, 128, 4, NULL, 0, 4, NULL, 0, 0, NULL, 0, NULL) == 0
+    assert s(NULL, 0, NULL, 3, 128, 4, NULL, 2, 2, NULL, 0, 0, NULL, 0, NULL) == 0
+
+
+def test_index_validation(L):
+    f = _fake()
+    sel = L.csa_index_select
+    # k out of range, Hi out of range, m out of range, missing scale, small workspace
+    assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 4, 100, 0, f, NULL, f, 1 << 20, NULL) == 3
+    assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 4, 100, 4096, f, NULL, f, 1 << 20, NULL) == 3
+    assert sel(f, f, f, f, 2, 17, f, 0, NULL, 0, 0, 4, 100, 16, f, NULL, f, 1 << 20, NULL) == 3
+    assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 0, 100, 16, f, NULL, f, 1 << 20, NULL) == 3
+    assert sel(f, f, f, f, 2, 8, f, 1, NULL, 0, 0, 4, 100, 16, f, NULL, f, 1 << 20, NULL) == 1
+    assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 4, 100, 16, f, NULL, f, 300, NULL) == 4
+    assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 4, 100, 16, NULL, NULL, f, 1 << 20, NULL) == 1
+    assert sel(f, f, f, f, 2, 8, f, 0, NULL, 12, 0, 4, 100, 16, f, NULL, f, 1 << 20, NULL) == 8
+    need = csa.csa_index_workspace_size(2, 512, 8, 16, 100)
+    assert need > 256
+    q = L.csa_index_query
+    assert q(f, 2, 100, 64, 8, f, f, f, f, f, f, 1 << 20, NULL) == 3          # D % 8
+    assert q(f, 2, 128, 64, 0, f, f, f, f, f, f, 1 << 20, NULL) == 3          # Hi
+    assert q(f, 2, 128, 64, 8, f, f, f, f, f, f, 256, NULL) == 4              # workspace
+
+
+def test_attend_validation(L):
+    f = _fake()
+    a = L.csa_sparse_attend
+    assert a(f, f, f, 2, 40, f, 0, f, 0, 4, f, 16, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 3   # H
+    assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 16, 2000, 0.1, f, NULL, f, 1 << 24, NULL) == 3  # W
+    assert a(f, f, f, 2, 64, f, 0, f, 0, 4, NULL, 16, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 1
+    assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 0, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 3
+    assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 16, 128, float("inf"), f, NULL, f, 1 << 24, NULL) == 2
+    assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 16, 128, 0.1, f, NULL, f, 1000, NULL) == 4
+    h = L.hca_attend
+    assert h(f, f, f, 2, 64, f, 0, f, 0, 128, -1, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 2
+    assert csa.csa_attend_workspace_size(8, 64, 1152) >= 8 * 9 * 64 * 130 * 4
+
+
+def test_library_calls_no_allocator():
+    """The library's sources call no device or host allocator (scratch is
+    the caller's workspace)."""
+    import pathlib
+    for src in sorted((pathlib.Path(csa.__file__).parent / "csrc").glob("*.cu")):
+        text = src.read_text()
+        for bad in ("cudaMalloc", "cudaFree", "cudaHostAlloc", "malloc("):
+            assert bad not in text, (src.name, bad)

@@ -1,0 +1,351 @@
+"""GPU parity of every C-ABI call against the CPU oracle, stage by stage.
+
+Each call is fed the oracle's outputs of the previous stage (so a stage is
+judged on identical inputs), at sizes that span several tiles, chunks and
+splits with ragged tails.  Tolerances: tests/gpu_cases.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_03_b200 import csa
+from tests.gpu_cases import (check_attention, check_compress_bf16, check_scores, check_topk, dev_bf16, dev_i32,
+                             host_bits, score_scale)
+from tests.pins import bf16_bits_to_f64, rand_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    csa.lib()
+
+
+# ---------------------------------------------------------------- compress
+@pytest.mark.parametrize("d,m,fmt", [(128, 4, 0), (128, 128, 0), (64, 4, 0), (64, 4, 1), (128, 1, 0), (64, 16, 1),
+                                     (128, 256, 0)])
+def test_compress(oracle, d, m, fmt):
+    rng = np.random.default_rng(100 + m + d + fmt)
+    B = 3
+    L = m * 70 + 3
+    raw = rand_bf16(rng, (B, L, d))
+    lens = np.array([L, L - m - 2, m * 3 + 1], np.int32)
+    z = rng.standard_normal((m, d)).astype(np.float32)
+    nmax = L // m
+    ref, ref_s = oracle.compress(raw, lens, z, 0, 1 << 30, out_fmt=fmt)
+    canary = 0x5A
+    if fmt == 0:
+        out = torch.full((B, nmax + 2, d), 0, dtype=torch.int16, device="cuda")
+        out.view(torch.uint8).fill_(canary)
+        out = out.view(torch.bfloat16)
+        scale = None
+    else:
+        out = torch.full((B, nmax + 2, d), canary, dtype=torch.uint8, device="cuda")
+        scale = torch.full((B, nmax + 2), -7.0, dtype=torch.float32, device="cuda")
+    csa.csa_compress(dev_bf16(raw), dev_i32(lens), torch.from_numpy(z).cuda(), m, 0, 1 << 30, out, fmt, scale)
+    torch.cuda.synchronize()
+    a = oracle.pool_weights(z)
+    for b in range(B):
+        nb = lens[b] // m
+        if fmt == 0:
+            g = host_bits(out[b])
+            x = bf16_bits_to_f64(raw[b, :nb * m]).reshape(nb, m, d)
+            absum = np.einsum("jid,id->jd", np.abs(x), np.abs(a))
+            check_compress_bf16(g[:nb], ref[b, :nb], exact=(m == 1), absum=absum, m=m)
+            assert (g[nb:].view(np.uint8) == canary).all(), "wrote past the complete blocks"
+        else:
+            g = out[b].cpu().numpy()
+            gs = scale[b].cpu().numpy()
+            assert (g[nb:] == canary).all() and (gs[nb:] == -7.0).all()
+            rs = ref_s[b, :nb]
+            rel = np.abs(gs[:nb] - rs) / rs
+            assert (rel <= 2 ** -7).all()
+            same = gs[:nb] == rs
+            dc = np.abs(g[:nb].astype(np.int32) - ref[b, :nb].astype(np.int32))
+            assert (dc[same] <= 1).all(), "E4M3 code more than one step off"
+            assert np.count_nonzero(dc) <= 0.01 * dc.size + 2
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_compress_exact_pooling_bit_exact(oracle, fmt):
+    """One-hot weights make pooling exact: bf16 rows and E4M3 codes/scales
+    must then match the oracle bit for bit."""
+    rng = np.random.default_rng(7)
+    m, d, B, L = 4, (128 if fmt == 0 else 64), 2, 4 * 300
+    raw = rand_bf16(rng, (B, L, d), scale=3.0)
+    lens = np.array([L, L - 9], np.int32)
+    z = np.full((m, d), -np.inf, np.float32)
+    z[2] = 0.0
+    ref, ref_s = oracle.compress(raw, lens, z, 0, 1 << 30, out_fmt=fmt)
+    N = L // m
+    if fmt == 0:
+        out = torch.zeros((B, N, d), dtype=torch.bfloat16, device="cuda")
+        scale = None
+    else:
+        out = torch.zeros((B, N, d), dtype=torch.uint8, device="cuda")
+        scale = torch.zeros((B, N), dtype=torch.float32, device="cuda")
+    csa.csa_compress(dev_bf16(raw), dev_i32(lens), torch.from_numpy(z).cuda(), m, 0, N, out, fmt, scale)
+    torch.cuda.synchronize()
+    for b in range(B):
+        nb = lens[b] // m
+        g = host_bits(out[b]) if fmt == 0 else out[b].cpu().numpy()
+        assert np.array_equal(g[:nb], ref[b, :nb])
+        if fmt == 1:
+            assert np.array_equal(scale[b, :nb].cpu().numpy(), ref_s[b, :nb])
+
+
+def test_compress_relative_range(oracle):
+    """blk_lo = -1 refreshes only the newest complete block of each sequence."""
+    rng = np.random.default_rng(8)
+    m, d, B, L = 4, 128, 3, 64
+    raw = rand_bf16(rng, (B, L, d))
+    lens = np.array([64, 63, 10], np.int32)
+    z = rng.standard_normal((m, d)).astype(np.float32)
+    full, _ = oracle.compress(raw, lens, z, 0, 1 << 30)
+    out = torch.zeros((B, 16, d), dtype=torch.bfloat16, device="cuda")
+    csa.csa_compress(dev_bf16(raw), dev_i32(lens), torch.from_numpy(z).cuda(), m, -1, 1, out)
+    g = host_bits(out)
+    for b in range(B):
+        nb = lens[b] // m
+        check_compress_bf16(g[b, nb - 1:nb], full[b, nb - 1:nb])
+        assert (g[b, :nb - 1] == 0).all() and (g[b, nb:] == 0).all()
+
+
+# ---------------------------------------------------------------- indexer
+@pytest.mark.parametrize("T,D,r,Hi", [(1, 1024, 256, 4), (8, 4096, 512, 8), (5, 512, 64, 16), (33, 256, 32, 3)])
+def test_index_query(oracle, T, D, r, Hi):
+    rng = np.random.default_rng(T + D + Hi)
+    h = rand_bf16(rng, (T, D))
+    W_dq = rand_bf16(rng, (r, D), D ** -0.5)
+    W_uq = rand_bf16(rng, (Hi * 64, r), r ** -0.5)
+    W_w = rand_bf16(rng, (Hi, D), D ** -0.5)
+    rq, rw = oracle.index_query(h, W_dq, W_uq, W_w)
+    q = torch.empty((T, Hi, 64), dtype=torch.float32, device="cuda")
+    w = torch.empty((T, Hi), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_index_workspace_size(T, r, Hi, 1, 1))
+    csa.csa_index_query(dev_bf16(h), dev_bf16(W_dq), dev_bf16(W_uq), dev_bf16(W_w), q, w, ws)
+    gq, gw = q.cpu().numpy().astype(np.float64), w.cpu().numpy().astype(np.float64)
+    for t in range(T):
+        assert np.abs(gq[t] - rq[t]).max() <= 1e-5 * np.abs(rq[t]).max()
+        assert np.abs(gw[t] - rw[t]).max() <= 1e-5 * np.abs(rw[t]).max()
+
+
+def _index_case(oracle, rng, B, N, Hi, T, fmt, m=4, ties=False, neg_w=False):
+    raw = rand_bf16(rng, (B, N * m, 64))
+    if ties:   # duplicate key rows -> exactly equal scores
+        raw[:, m * 10:m * 40] = raw[:, :m * 30]
+    z = rng.standard_normal((m, 64)).astype(np.float32)
+    lens = np.full(B, N * m, np.int32)
+    keys, kscale = oracle.compress(raw, lens, z, 0, 1 << 30, out_fmt=fmt)
+    q = rng.standard_normal((T, Hi, 64)).astype(np.float32)
+    w = rng.standard_normal((T, Hi)).astype(np.float32)
+    if neg_w:
+        w = -np.abs(w)
+    q_seq = rng.integers(0, B, T).astype(np.int32)
+    q_pos = rng.integers(0, N * m, T).astype(np.int32)
+    q_pos[0] = N * m - 1
+    if T > 1:
+        q_pos[1] = 2     # V = 0 for m = 4
+    return keys, kscale, q, w, q_seq, q_pos
+
+
+def _keys_f64(oracle, keys, kscale, fmt):
+    if fmt == 0:
+        return bf16_bits_to_f64(keys)
+    return oracle.e4m3_decode(keys) * kscale[..., None].astype(np.float64)
+
+
+@pytest.mark.parametrize("fmt,Hi,N,T", [(0, 8, 5000, 6), (1, 8, 5000, 6), (0, 4, 1024, 1), (0, 16, 3000, 4),
+                                        (1, 3, 2100, 3)])
+def test_index_scores(oracle, fmt, Hi, N, T):
+    rng = np.random.default_rng(fmt * 10 + Hi + N)
+    m = 4
+    keys, ks, q, w, q_seq, q_pos = _index_case(oracle, rng, 2, N, Hi, T, fmt)
+    ref = oracle.index_scores(q.astype(np.float64), w.astype(np.float64), q_seq, q_pos, keys, m, N, kidx_fmt=fmt,
+                              kidx_scale=ks)
+    kd = torch.from_numpy(keys).cuda() if fmt == 1 else dev_bf16(keys)
+    out = torch.empty((T, N), dtype=torch.float32, device="cuda")
+    csa.csa_index_scores(torch.from_numpy(q).cuda(), torch.from_numpy(w).cuda(), dev_i32(q_seq), dev_i32(q_pos), kd, m,
+                         N, out, kidx_scale=None if ks is None else torch.from_numpy(ks).cuda())
+    g = out.cpu().numpy()
+    kf = _keys_f64(oracle, keys, ks, fmt)
+    for t in range(T):
+        A = score_scale(q[t].astype(np.float64), w[t].astype(np.float64), kf[q_seq[t]])
+        check_scores(g[t], ref[t], A)
+
+
+@pytest.mark.parametrize("fmt,Hi,N,T,k,ties,neg", [
+    (0, 8, 5000, 6, 64, False, False), (0, 8, 9000, 3, 512, False, False), (1, 8, 9000, 3, 512, False, False),
+    (0, 4, 1024, 1, 64, False, False), (0, 8, 3000, 4, 2048, False, False), (0, 8, 2500, 5, 1, False, False),
+    (0, 8, 4000, 4, 100, True, False), (0, 8, 4000, 4, 300, False, True), (1, 16, 20000, 2, 1024, False, False)])
+def test_index_select(oracle, fmt, Hi, N, T, k, ties, neg):
+    rng = np.random.default_rng(1000 + fmt + Hi + N + k)
+    m = 4
+    keys, ks, q, w, q_seq, q_pos = _index_case(oracle, rng, 2, N, Hi, T, fmt, ties=ties, neg_w=neg)
+    S = oracle.index_scores(q.astype(np.float64), w.astype(np.float64), q_seq, q_pos, keys, m, N, kidx_fmt=fmt,
+                            kidx_scale=ks)
+    kd = torch.from_numpy(keys).cuda() if fmt == 1 else dev_bf16(keys)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_index_workspace_size(T, 0, Hi, k, N))
+    csa.csa_index_select(torch.from_numpy(q).cuda(), torch.from_numpy(w).cuda(), dev_i32(q_seq), dev_i32(q_pos), kd, m,
+                         N, k, idx, sc, ws, kidx_scale=None if ks is None else torch.from_numpy(ks).cuda())
+    ws.check()
+    gi, gs = idx.cpu().numpy(), sc.cpu().numpy()
+    kf = _keys_f64(oracle, keys, ks, fmt)
+    for t in range(T):
+        V = min((q_pos[t] + 1) // m, N)
+        A = score_scale(q[t].astype(np.float64), w[t].astype(np.float64), kf[q_seq[t]])
+        check_topk(gi[t], gs[t], S[t], A, V, k)
+
+
+def test_index_topk_from_hidden_state(oracle):
+    """csa_index_topk (projection + selection) against the oracle chain."""
+    rng = np.random.default_rng(55)
+    T, D, r, Hi, N, k, m = 4, 1024, 256, 8, 6000, 256, 4
+    keys, _, _, _, q_seq, q_pos = _index_case(oracle, rng, 2, N, Hi, T, 0)
+    h = rand_bf16(rng, (T, D))
+    W_dq = rand_bf16(rng, (r, D), D ** -0.5)
+    W_uq = rand_bf16(rng, (Hi * 64, r), r ** -0.5)
+    W_w = rand_bf16(rng, (Hi, D), D ** -0.5)
+    rq, rw = oracle.index_query(h, W_dq, W_uq, W_w)
+    S = oracle.index_scores(rq, rw, q_seq, q_pos, keys, m, N)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_index_workspace_size(T, r, Hi, k, N))
+    csa.csa_index_topk(dev_bf16(h), dev_bf16(W_dq), dev_bf16(W_uq), dev_bf16(W_w), dev_i32(q_seq), dev_i32(q_pos),
+                       dev_bf16(keys), m, N, k, idx, sc, ws)
+    kf = bf16_bits_to_f64(keys)
+    for t in range(T):
+        V = min((q_pos[t] + 1) // m, N)
+        A = score_scale(rq[t], rw[t], kf[q_seq[t]])
+        check_topk(idx[t].cpu().numpy(), sc[t].cpu().numpy(), S[t], A, V, k)
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(rng, B, N, L, H, T, k, W, m):
+    q = rand_bf16(rng, (T, H, 128))
+    comp = rand_bf16(rng, (B, N, 128))
+    raw = rand_bf16(rng, (B, L, 128))
+    q_seq = rng.integers(0, B, T).astype(np.int32)
+    q_pos = rng.integers(0, min(L, N * m), T).astype(np.int32)
+    q_pos[0] = min(L, N * m) - 1
+    if T > 2:
+        q_pos[1] = 1
+        q_pos[2] = W + 3
+    idx = np.full((T, k), -1, np.int32)
+    for t in range(T):
+        V = (q_pos[t] + 1) // m
+        n = min(k, V)
+        if n:
+            sel = rng.choice(V, n, replace=False).astype(np.int32)
+            sel[rng.random(n) < 0.05] = -1      # scattered padding entries
+            idx[t, :n] = sel
+    return q, comp, raw, q_seq, q_pos, idx
+
+
+@pytest.mark.parametrize("H,k,W,T", [(64, 512, 128, 5), (16, 64, 128, 3), (128, 200, 0, 3), (64, 1024, 128, 2),
+                                     (32, 37, 5, 4), (48, 300, 1024, 3)])
+def test_sparse_attend(oracle, H, k, W, T):
+    rng = np.random.default_rng(H + k + W)
+    m, B, N = 4, 2, 2000
+    L = N * m + 3
+    q, comp, raw, q_seq, q_pos, idx = _attn_case(rng, B, N, L, H, T, k, W, m)
+    scale = 128 ** -0.5
+    ref, rlse = oracle.sparse_attend(q, q_seq, q_pos, comp, raw, m, idx, W, scale)
+    out = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_attend_workspace_size(T, H, k + W))
+    csa.csa_sparse_attend(dev_bf16(q), dev_i32(q_seq), dev_i32(q_pos), dev_bf16(comp), dev_bf16(raw), m,
+                          dev_i32(idx), W, scale, out, lse, ws)
+    ws.check()
+    check_attention(bf16_bits_to_f64(host_bits(out)), lse.cpu().numpy().astype(np.float64), ref, rlse)
+
+
+@pytest.mark.parametrize("H,W,T,mp", [(64, 128, 4, 128), (16, 0, 3, 128), (64, 128, 3, 16)])
+def test_hca_attend(oracle, H, W, T, mp):
+    rng = np.random.default_rng(H + W + mp)
+    B, L = 2, 128 * 130 + 5
+    N = L // mp
+    q = rand_bf16(rng, (T, H, 128))
+    comp = rand_bf16(rng, (B, N, 128))
+    raw = rand_bf16(rng, (B, L, 128))
+    q_seq = rng.integers(0, B, T).astype(np.int32)
+    q_pos = rng.integers(0, L, T).astype(np.int32)
+    q_pos[0] = L - 1
+    q_pos[1] = 5
+    scale = 0.09
+    ref, rlse = oracle.hca_attend(q, q_seq, q_pos, comp, raw, mp, W, scale)
+    out = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_attend_workspace_size(T, H, N + W))
+    csa.hca_attend(dev_bf16(q), dev_i32(q_seq), dev_i32(q_pos), dev_bf16(comp), dev_bf16(raw), mp, N, W, scale, out,
+                   lse, ws)
+    check_attention(bf16_bits_to_f64(host_bits(out)), lse.cpu().numpy().astype(np.float64), ref, rlse)
+
+
+def test_attend_empty_set_and_bad_index(oracle):
+    """Nothing visible -> out 0, lse -inf; an index past V(t) is skipped and
+    flagged in the workspace status word (no trap)."""
+    rng = np.random.default_rng(3)
+    H, m, N, L = 16, 4, 64, 256
+    q = rand_bf16(rng, (2, H, 128))
+    comp = rand_bf16(rng, (1, N, 128))
+    raw = rand_bf16(rng, (1, L, 128))
+    idx = np.array([[-1, -1, -1], [3, 60, 1]], np.int32)      # query 1: V = 11, index 60 is invalid
+    q_pos = np.array([2, 45], np.int32)
+    out = torch.empty((2, H, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((2, H), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_attend_workspace_size(2, H, 3))
+    csa.csa_sparse_attend(dev_bf16(q), dev_i32([0, 0]), dev_i32(q_pos), dev_bf16(comp), dev_bf16(raw), m,
+                          dev_i32(idx), 0, 0.1, out, lse, ws)
+    with pytest.raises(csa.CsaError) as e:
+        ws.check()
+    assert e.value.status == 7
+    ws.check()   # cleared
+    o = out.float().cpu().numpy()
+    assert (o[0] == 0).all() and np.isneginf(lse[0].cpu().numpy()).all()
+    ref, rlse = oracle.sparse_attend(q[1:], [0], q_pos[1:], comp, raw, m, idx[1:], 0, 0.1)
+    check_attention(o[1:], lse[1:].cpu().numpy(), ref, rlse)
+
+
+# ---------------------------------------------------------------- invariance
+def test_batch_invariance_and_determinism(oracle):
+    """A query's top-k and attention output are bitwise the same alone and
+    inside a batch (which changes the chunking), and across reruns."""
+    rng = np.random.default_rng(77)
+    m, N, Hi, k, H, W = 4, 12000, 8, 512, 64, 128
+    B = 6
+    keys, _, q, w, q_seq, q_pos = _index_case(oracle, rng, B, N, Hi, B, 0)
+    q_seq = np.arange(B, dtype=np.int32)
+    q_pos = np.full(B, N * m - 1, np.int32)
+    comp = rand_bf16(rng, (B, N, 128))
+    raw = rand_bf16(rng, (B, N * m, 128))
+    qa = rand_bf16(rng, (B, H, 128))
+    kd, cd, rd = dev_bf16(keys), dev_bf16(comp), dev_bf16(raw)
+
+    def run(sel):
+        T = len(sel)
+        idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+        sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+        ws = csa.Workspace(csa.csa_index_workspace_size(T, 0, Hi, k, N))
+        csa.csa_index_select(torch.from_numpy(q[sel]).cuda(), torch.from_numpy(w[sel]).cuda(), dev_i32(q_seq[sel]),
+                             dev_i32(q_pos[sel]), kd, m, N, k, idx, sc, ws)
+        out = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((T, H), dtype=torch.float32, device="cuda")
+        wa = csa.Workspace(csa.csa_attend_workspace_size(T, H, k + W))
+        csa.csa_sparse_attend(dev_bf16(qa[sel]), dev_i32(q_seq[sel]), dev_i32(q_pos[sel]), cd, rd, m, idx, W,
+                              128 ** -0.5, out, lse, wa)
+        torch.cuda.synchronize()
+        return idx.cpu().numpy(), sc.cpu().numpy(), host_bits(out), lse.cpu().numpy()
+
+    full = run(np.arange(B))
+    again = run(np.arange(B))
+    for a, b in zip(full, again):
+        assert np.array_equal(a, b, equal_nan=True)
+    for t in (0, 3, 5):
+        alone = run(np.array([t]))
+        for a, b in zip(full, alone):
+            assert np.array_equal(a[t], b[0], equal_nan=True)
