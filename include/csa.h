@@ -97,6 +97,7 @@ enum { CSA_DEV_BAD_INDEX = 1u, CSA_DEV_TIMEOUT = 2u };
 #define CSA_MAX_HI 16      /* indexer heads: 1..16 */
 #define CSA_MAX_K 2048     /* top-k: 1..2048 */
 #define CSA_MAX_W 1024     /* window: 0..1024 */
+#define CSA_MAX_D 7168     /* indexer d_model and rank: multiples of 8 up to this */
 /* attention heads H: 16, 32, 48, ..., 128 (a multiple of 16) */
 
 /* Human-readable name of a status code (static string). */
@@ -163,7 +164,7 @@ CSA_API size_t csa_index_workspace_size(int T, int r, int Hi, int k, int max_blo
  * Indexer query projection.  h bf16 [T][D]; W_dq bf16 [r][D]; W_uq bf16
  * [Hi*64][r]; W_w bf16 [Hi][D].  Outputs q fp32 [T][Hi][64] and w fp32 [T][Hi]
  * (not rounded further).  u = W_dq h is kept in fp32 (workspace).
- * Constraints: D % 8 == 0, r % 8 == 0, 1 <= Hi <= 16.
+ * Constraints: D % 8 == 0, r % 8 == 0, D, r <= CSA_MAX_D, 1 <= Hi <= 16.
  */
 CSA_API csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
                            const void* W_dq, const void* W_uq, const void* W_w,
@@ -187,10 +188,11 @@ CSA_API csa_status csa_index_scores(const float* q, const float* w, const int32_
  * Score every visible block and select the per-query top-k (R5): out_idx
  * int32 [T][k] sorted by (score desc, index asc), padded with -1;
  * out_score fp32 [T][k] (NaN at padding) or NULL.  max_blocks bounds V(t)
- * for every query (blocks past it are ignored).  The scores are never
- * materialised: each CTA keeps its chunk's scores on chip and emits its
- * exact local top-k, which later stages merge.  Equivalent to
- * csa_index_stage_score followed by csa_index_stage_merge.
+ * for every query (blocks past it are ignored).  The fp32 scores and a
+ * 2048-bin histogram of 32-key maxima go to the workspace;
+ * the selection then only touches the scores at or above the k-th key's
+ * bin.  Equivalent to csa_index_stage_score followed by
+ * csa_index_stage_merge.
  */
 CSA_API csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq,
                             const int32_t* q_pos, int T, int Hi,
@@ -201,7 +203,7 @@ CSA_API csa_status csa_index_select(const float* q, const float* w, const int32_
                             void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* First stage of csa_index_select: the streaming score kernel, writing the
- * per-chunk exact top-k candidates into the workspace. */
+ * scores and their key histogram into the workspace. */
 CSA_API csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* q_seq,
                                  const int32_t* q_pos, int T, int Hi,
                                  const void* kidx, int kidx_fmt, const float* kidx_scale,
@@ -209,11 +211,13 @@ CSA_API csa_status csa_index_stage_score(const float* q, const float* w, const i
                                  int m, int max_blocks, int k,
                                  void* ws, size_t ws_bytes, csa_stream_t stream);
 
-/* Second stage: merge the candidates left in the workspace by
- * csa_index_stage_score (same T, max_blocks, k) into out_idx / out_score. */
-CSA_API csa_status csa_index_stage_merge(int T, int max_blocks, int k,
-                                 int32_t* out_idx, float* out_score,
-                                 void* ws, size_t ws_bytes, csa_stream_t stream);
+/* Second stage: from the scores and histogram left in the workspace by
+ * csa_index_stage_score (same T, m, max_blocks and workspace), collect the
+ * candidates at or above the k-th largest key's histogram bin and write the
+ * exact sorted top-k to out_idx / out_score. */
+CSA_API csa_status csa_index_stage_merge(const int32_t* q_pos, int T, int m, int max_blocks, int k,
+                                         int32_t* out_idx, float* out_score,
+                                         void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* csa_index_query followed by csa_index_select. */
 CSA_API csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq,
@@ -230,9 +234,11 @@ CSA_API csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq,
 /*    dense over all visible compressed rows + window).  Reading R6.      */
 /* ------------------------------------------------------------------ */
 
-/* Workspace for csa_sparse_attend (max_rows = k + W) and hca_attend
- * (max_rows = max_blocks + W). */
+/* Workspace for csa_sparse_attend (max_rows = k + W). */
 CSA_API size_t csa_attend_workspace_size(int T, int H, int max_rows);
+
+/* Workspace for hca_attend (max_rows = max_blocks + W). */
+CSA_API size_t hca_attend_workspace_size(int T, int H, int max_rows);
 
 /*
  * q bf16 [T][H][128]; comp bf16 compressed latent rows [B][.][128] (row j at
@@ -241,8 +247,8 @@ CSA_API size_t csa_attend_workspace_size(int T, int H, int max_rows);
  * are skipped and flagged CSA_DEV_BAD_INDEX).  out bf16 [T][H][128];
  * lse fp32 [T][H] (natural log of the softmax denominator, -inf for an
  * empty set) or NULL.  An empty attended set gives out = 0.
- * fp32 logits, softmax and accumulation; split-K over fixed 128-row
- * splits merged in a fixed order.
+ * fp32 logits, softmax and accumulation; split-K over fixed 64-row splits
+ * (512-row for hca_attend) merged in a fixed order.
  */
 CSA_API csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
                              int T, int H, const void* comp, int64_t comp_seq_stride,

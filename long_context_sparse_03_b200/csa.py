@@ -47,10 +47,11 @@ _SIGS = {
     "csa_index_scores": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _P, _P]),
     "csa_index_select": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _I, _P, _P, _P, _S, _P]),
     "csa_index_stage_score": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _I, _P, _S, _P]),
-    "csa_index_stage_merge": (_I, [_I, _I, _I, _P, _P, _P, _S, _P]),
+    "csa_index_stage_merge": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _S, _P]),
     "csa_index_topk": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _L, _L, _I, _I, _I, _P, _P,
                             _P, _S, _P]),
     "csa_attend_workspace_size": (_S, [_I, _I, _I]),
+    "hca_attend_workspace_size": (_S, [_I, _I, _I]),
     "csa_sparse_attend": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _P, _I, _I, _F, _P, _P, _P, _S, _P]),
     "hca_attend": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _I, _I, _F, _P, _P, _P, _S, _P]),
 }
@@ -134,6 +135,10 @@ def csa_attend_workspace_size(T, H, max_rows) -> int:
     return int(lib().csa_attend_workspace_size(T, H, max_rows))
 
 
+def hca_attend_workspace_size(T, H, max_rows) -> int:
+    return int(lib().hca_attend_workspace_size(T, H, max_rows))
+
+
 # ---------------------------------------------------------------- calls
 def csa_compress(raw, lens, pool_logits, m, blk_lo, blk_hi, out, out_fmt=FMT_BF16, out_scale=None,
                  stream=None):
@@ -191,9 +196,10 @@ def csa_index_stage_score(q, w, q_seq, q_pos, kidx, m, max_blocks, k, ws: Worksp
     _check(st, "csa_index_stage_score")
 
 
-def csa_index_stage_merge(T, max_blocks, k, out_idx, out_score, ws: Workspace, stream=None):
-    st = lib().csa_index_stage_merge(T, max_blocks, k, _ptr(out_idx), _ptr(out_score), ws.ptr(), ws.nbytes,
-                                     _stream(stream))
+def csa_index_stage_merge(q_pos, m, max_blocks, k, out_idx, out_score, ws: Workspace, stream=None):
+    T = int(q_pos.shape[0])
+    st = lib().csa_index_stage_merge(_ptr(q_pos), T, m, max_blocks, k, _ptr(out_idx), _ptr(out_score), ws.ptr(),
+                                     ws.nbytes, _stream(stream))
     _check(st, "csa_index_stage_merge")
 
 

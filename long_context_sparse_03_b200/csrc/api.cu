@@ -20,19 +20,16 @@ cudaError_t launch_compress(const void* raw, int64_t raw_stride, const int* lens
 cudaError_t launch_index_query(const void* h, int T, int D, int r, int Hi, const void* W_dq, const void* W_uq,
                                const void* W_w, float* q_out, float* w_out, float* u_ws, cudaStream_t stream,
                                int* launches);
-struct SelectPlan {
-    int chunk, nchunks, kc;
-    int64_t n0;
-    size_t cand_a, cand_b;
-};
-SelectPlan plan_select(int T, int max_blocks, int k);
 cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
-                               const void* kidx, int fmt, const float* kscale, int64_t kstride_elems,
-                               int64_t sstride, int m, int max_blocks, int k, uint64_t* cand, float* scores,
-                               cudaStream_t stream, int* launches);
-cudaError_t launch_index_merge(int T, int max_blocks, int k, uint64_t* cand_a, uint64_t* cand_b, int* out_idx,
-                               float* out_score, cudaStream_t stream, int* launches);
-int attend_nsplit(int max_rows);
+                               const void* kidx, int fmt, const float* kscale, int64_t kstride_elems, int64_t sstride,
+                               int m, int max_blocks, int k, float* scores, int64_t ld_scores, unsigned* hist,
+                               unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream, int* launches);
+cudaError_t launch_index_select_tail(const float* scores, int64_t ld_scores, const unsigned* thr, const int* q_pos,
+                                     int T, int m, int max_blocks, int k, uint64_t* cand, int64_t cand_cap,
+                                     unsigned* cnt, int* out_idx, float* out_score, cudaStream_t stream,
+                                     int* launches);
+constexpr int kHistBins = 2048;
+int attend_nsplit(int max_rows, bool dense);
 cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int T, int H, const void* comp,
                           int64_t comp_stride, const void* raw, int64_t raw_stride, int m, const int* idx, int k,
                           int max_blocks, int W, float scale, void* out, float* lse, float* part_o,
@@ -69,10 +66,15 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
     } while (0)
 
 // ---------------------------------------------------------------- layouts
+// candidate rows start 16-byte aligned (the rank pass stages them with cp.async)
+int64_t cand_cap(int max_blocks) { return ((int64_t)max_blocks + 1) & ~(int64_t)1; }
+
 struct IndexLayout {
-    size_t u, q, w, cand_a, cand_b, total;
+    size_t u, q, w, hist, cnt, done, thr, scores, cand, total;
 };
-IndexLayout index_layout(int T, int r, int Hi, int k, int max_blocks) {
+// header | u [T][r] | q [T][Hi][64] | w [T][Hi] | hist [T][4096] | cnt [T] |
+// done [T] | thr [T] | scores [T][max_blocks] fp32 | cand [T][max_blocks] u64
+IndexLayout index_layout(int T, int r, int Hi, int max_blocks) {
     IndexLayout L;
     size_t off = CSA_WS_HEADER_BYTES;
     L.u = off;
@@ -81,11 +83,15 @@ IndexLayout index_layout(int T, int r, int Hi, int k, int max_blocks) {
     off = up256(off + (size_t)T * Hi * 64 * 4);
     L.w = off;
     off = up256(off + (size_t)T * Hi * 4);
-    csa::SelectPlan p = csa::plan_select(T, max_blocks > 0 ? max_blocks : 1, k > 0 ? k : 1);
-    L.cand_a = off;
-    off = up256(off + p.cand_a);
-    L.cand_b = off;
-    off = up256(off + p.cand_b);
+    L.hist = off;
+    L.cnt = off + (size_t)T * csa::kHistBins * 4;
+    L.done = L.cnt + (size_t)T * 4;
+    L.thr = L.done + (size_t)T * 4;
+    off = up256(L.thr + (size_t)T * 4);
+    L.scores = off;
+    off = up256(off + (size_t)T * max_blocks * 4);
+    L.cand = off;
+    off = up256(off + (size_t)T * cand_cap(max_blocks) * 8);
     L.total = off;
     return L;
 }
@@ -93,9 +99,9 @@ IndexLayout index_layout(int T, int r, int Hi, int k, int max_blocks) {
 struct AttendLayout {
     size_t part_o, part_ml, total;
 };
-AttendLayout attend_layout(int T, int H, int max_rows) {
+AttendLayout attend_layout(int T, int H, int max_rows, bool dense) {
     AttendLayout L;
-    const int ns = csa::attend_nsplit(max_rows);
+    const int ns = csa::attend_nsplit(max_rows, dense);
     size_t off = CSA_WS_HEADER_BYTES;
     L.part_o = off;
     off = up256(off + (size_t)T * ns * H * 128 * 4);
@@ -197,8 +203,9 @@ csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* 
 
 // ---------------------------------------------------------------- indexer
 size_t csa_index_workspace_size(int T, int r, int Hi, int k, int max_blocks) {
-    if (T < 0 || r < 0 || Hi < 0) return 0;
-    return index_layout(T, r, Hi, k, max_blocks).total;
+    (void)k;
+    if (T < 0 || r < 0 || Hi < 0 || max_blocks < 0) return 0;
+    return index_layout(T, r, Hi, max_blocks).total;
 }
 
 csa_status csa_index_query(const void* h, int T, int D, int r, int Hi, const void* W_dq, const void* W_uq,
@@ -206,6 +213,7 @@ csa_status csa_index_query(const void* h, int T, int D, int r, int Hi, const voi
                            csa_stream_t stream) {
     REQUIRE(T >= 0 && D >= 8 && r >= 8, CSA_ERR_SHAPE, "T = %d, D = %d, r = %d", T, D, r);
     REQUIRE(D % 8 == 0 && r % 8 == 0, CSA_ERR_UNSUPPORTED, "D and r must be multiples of 8");
+    REQUIRE(D <= CSA_MAX_D && r <= CSA_MAX_D, CSA_ERR_UNSUPPORTED, "D and r must be <= %d", CSA_MAX_D);
     REQUIRE(Hi >= 1 && Hi <= CSA_MAX_HI, CSA_ERR_UNSUPPORTED, "Hi = %d outside 1..%d", Hi, CSA_MAX_HI);
     if (T == 0) return ok();
     REQUIRE(h && W_dq && W_uq && W_w && q_out && w_out && ws, CSA_ERR_NULL, "a required pointer is NULL");
@@ -230,12 +238,48 @@ csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq
                                       scale_seq_stride, m, max_blocks);
     if (s != CSA_OK || T == 0) return s;
     REQUIRE(scores, CSA_ERR_NULL, "scores is NULL");
+    // invisible entries stay NaN (all-ones bytes)
+    cudaError_t e = cudaMemsetAsync(scores, 0xFF, (size_t)T * max_blocks * 4, (cudaStream_t)stream);
     int n = 0;
-    cudaError_t e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
-                                            scale_seq_stride, m, max_blocks, 1, nullptr, scores,
-                                            (cudaStream_t)stream, &n);
+    if (e == cudaSuccess)
+        e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
+                                    scale_seq_stride, m, max_blocks, 1, scores, max_blocks, nullptr, nullptr,
+                                    nullptr, nullptr, (cudaStream_t)stream, &n);
     count(n);
     if (e != cudaSuccess) return cuda_fail(e, "csa_index_scores");
+    return ok();
+}
+
+static csa_status stage_score(const char* who, const float* q, const float* w, const int32_t* q_seq,
+                              const int32_t* q_pos, int T, int Hi, const void* kidx, int kidx_fmt,
+                              const float* kidx_scale, int64_t kidx_seq_stride, int64_t scale_seq_stride, int m,
+                              int max_blocks, int k, const IndexLayout& L, void* ws, cudaStream_t stream) {
+    char* base = (char*)ws;
+    cudaError_t e = cudaMemsetAsync(base + L.hist, 0, L.scores - L.hist, stream);  // hist, cnt, done, thr
+    int n = 0;
+    if (e == cudaSuccess)
+        e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
+                                    scale_seq_stride, m, max_blocks, k, reinterpret_cast<float*>(base + L.scores),
+                                    max_blocks, reinterpret_cast<unsigned*>(base + L.hist),
+                                    reinterpret_cast<unsigned*>(base + L.done),
+                                    reinterpret_cast<unsigned*>(base + L.thr), reinterpret_cast<unsigned*>(base),
+                                    stream, &n);
+    count(n);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+    return ok();
+}
+
+static csa_status stage_merge(const char* who, const int32_t* q_pos, int T, int m, int max_blocks, int k,
+                              int32_t* out_idx, float* out_score, const IndexLayout& L, void* ws,
+                              cudaStream_t stream) {
+    char* base = (char*)ws;
+    int n = 0;
+    cudaError_t e = csa::launch_index_select_tail(
+        reinterpret_cast<const float*>(base + L.scores), max_blocks, reinterpret_cast<const unsigned*>(base + L.thr),
+        q_pos, T, m, max_blocks, k, reinterpret_cast<uint64_t*>(base + L.cand), cand_cap(max_blocks),
+        reinterpret_cast<unsigned*>(base + L.cnt), out_idx, out_score, stream, &n);
+    count(n);
+    if (e != cudaSuccess) return cuda_fail(e, who);
     return ok();
 }
 
@@ -250,35 +294,24 @@ csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* 
     if (T == 0) return ok();
     REQUIRE(ws, CSA_ERR_WORKSPACE, "ws is NULL");
     REQUIRE(aligned16(ws), CSA_ERR_ALIGN, "ws must be 16-byte aligned");
-    // the candidate buffers do not depend on r / Hi: size them with r = Hi = 0
-    IndexLayout L = index_layout(T, 0, 0, k, max_blocks);
+    IndexLayout L = index_layout(T, 0, 0, max_blocks);
     REQUIRE(ws_bytes >= L.total, CSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
-    int n = 0;
-    cudaError_t e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
-                                            scale_seq_stride, m, max_blocks, k,
-                                            reinterpret_cast<uint64_t*>((char*)ws + L.cand_a), nullptr,
-                                            (cudaStream_t)stream, &n);
-    count(n);
-    if (e != cudaSuccess) return cuda_fail(e, "csa_index_stage_score");
-    return ok();
+    return stage_score("csa_index_stage_score", q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale,
+                       kidx_seq_stride, scale_seq_stride, m, max_blocks, k, L, ws, (cudaStream_t)stream);
 }
 
-csa_status csa_index_stage_merge(int T, int max_blocks, int k, int32_t* out_idx, float* out_score, void* ws,
-                                 size_t ws_bytes, csa_stream_t stream) {
+csa_status csa_index_stage_merge(const int32_t* q_pos, int T, int m, int max_blocks, int k, int32_t* out_idx,
+                                 float* out_score, void* ws, size_t ws_bytes, csa_stream_t stream) {
     REQUIRE(T >= 0 && max_blocks >= 1, CSA_ERR_SHAPE, "T = %d, max_blocks = %d", T, max_blocks);
+    REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
     REQUIRE(k >= 1 && k <= CSA_MAX_K, CSA_ERR_UNSUPPORTED, "k = %d outside 1..%d", k, CSA_MAX_K);
     if (T == 0) return ok();
-    REQUIRE(out_idx, CSA_ERR_NULL, "out_idx is NULL");
+    REQUIRE(q_pos && out_idx, CSA_ERR_NULL, "q_pos and out_idx are required");
     REQUIRE(ws, CSA_ERR_WORKSPACE, "ws is NULL");
-    IndexLayout L = index_layout(T, 0, 0, k, max_blocks);
+    IndexLayout L = index_layout(T, 0, 0, max_blocks);
     REQUIRE(ws_bytes >= L.total, CSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
-    int n = 0;
-    cudaError_t e = csa::launch_index_merge(T, max_blocks, k, reinterpret_cast<uint64_t*>((char*)ws + L.cand_a),
-                                            reinterpret_cast<uint64_t*>((char*)ws + L.cand_b), out_idx, out_score,
-                                            (cudaStream_t)stream, &n);
-    count(n);
-    if (e != cudaSuccess) return cuda_fail(e, "csa_index_stage_merge");
-    return ok();
+    return stage_merge("csa_index_stage_merge", q_pos, T, m, max_blocks, k, out_idx, out_score, L, ws,
+                       (cudaStream_t)stream);
 }
 
 csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq, const int32_t* q_pos, int T,
@@ -289,7 +322,7 @@ csa_status csa_index_select(const float* q, const float* w, const int32_t* q_seq
     csa_status s = csa_index_stage_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
                                          scale_seq_stride, m, max_blocks, k, ws, ws_bytes, stream);
     if (s != CSA_OK) return s;
-    return csa_index_stage_merge(T, max_blocks, k, out_idx, out_score, ws, ws_bytes, stream);
+    return csa_index_stage_merge(q_pos, T, m, max_blocks, k, out_idx, out_score, ws, ws_bytes, stream);
 }
 
 csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq, const void* W_uq, const void* W_w,
@@ -303,35 +336,33 @@ csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq, const v
     REQUIRE(k >= 1 && k <= CSA_MAX_K, CSA_ERR_UNSUPPORTED, "k = %d outside 1..%d", k, CSA_MAX_K);
     REQUIRE(max_blocks >= 1, CSA_ERR_SHAPE, "max_blocks = %d < 1", max_blocks);
     if (T == 0) return ok();
+    REQUIRE(out_idx, CSA_ERR_NULL, "out_idx is NULL");
     REQUIRE(ws, CSA_ERR_WORKSPACE, "ws is NULL");
-    IndexLayout L = index_layout(T, r, Hi, k, max_blocks);
+    IndexLayout L = index_layout(T, r, Hi, max_blocks);
     REQUIRE(ws_bytes >= L.total, CSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
     float* qb = reinterpret_cast<float*>((char*)ws + L.q);
     float* wb = reinterpret_cast<float*>((char*)ws + L.w);
-    csa_status s = csa_index_query(h, T, D, r, Hi, W_dq, W_uq, W_w, qb, wb, ws, ws_bytes, stream);
-    if (s != CSA_OK) return s;
-    // scoring and merge use the candidate region that follows u / q / w
     csa_status c = check_index_common(qb, wb, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
                                       scale_seq_stride, m, max_blocks);
     if (c != CSA_OK) return c;
-    int n = 0;
-    cudaError_t e = csa::launch_index_score(qb, wb, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
-                                            scale_seq_stride, m, max_blocks, k,
-                                            reinterpret_cast<uint64_t*>((char*)ws + L.cand_a), nullptr,
-                                            (cudaStream_t)stream, &n);
-    if (e == cudaSuccess)
-        e = csa::launch_index_merge(T, max_blocks, k, reinterpret_cast<uint64_t*>((char*)ws + L.cand_a),
-                                    reinterpret_cast<uint64_t*>((char*)ws + L.cand_b), out_idx, out_score,
-                                    (cudaStream_t)stream, &n);
-    count(n);
-    if (e != cudaSuccess) return cuda_fail(e, "csa_index_topk");
-    return ok();
+    csa_status s = csa_index_query(h, T, D, r, Hi, W_dq, W_uq, W_w, qb, wb, ws, ws_bytes, stream);
+    if (s != CSA_OK) return s;
+    s = stage_score("csa_index_topk", qb, wb, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
+                    scale_seq_stride, m, max_blocks, k, L, ws, (cudaStream_t)stream);
+    if (s != CSA_OK) return s;
+    return stage_merge("csa_index_topk", q_pos, T, m, max_blocks, k, out_idx, out_score, L, ws,
+                       (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------- attention
 size_t csa_attend_workspace_size(int T, int H, int max_rows) {
     if (T < 0 || H < 0 || max_rows < 0) return 0;
-    return attend_layout(T, H, max_rows).total;
+    return attend_layout(T, H, max_rows, false).total;
+}
+
+size_t hca_attend_workspace_size(int T, int H, int max_rows) {
+    if (T < 0 || H < 0 || max_rows < 0) return 0;
+    return attend_layout(T, H, max_rows, true).total;
 }
 
 static csa_status attend_common(const char* who, const void* q, const int32_t* q_seq, const int32_t* q_pos, int T,
@@ -352,7 +383,7 @@ static csa_status attend_common(const char* who, const void* q, const int32_t* q
     REQUIRE(ws, CSA_ERR_WORKSPACE, "ws is NULL");
     REQUIRE(aligned16(ws), CSA_ERR_ALIGN, "ws must be 16-byte aligned");
     const int max_rows = (idx ? k : max_blocks) + W;
-    AttendLayout L = attend_layout(T, H, max_rows);
+    AttendLayout L = attend_layout(T, H, max_rows, idx == nullptr);
     REQUIRE(ws_bytes >= L.total, CSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
     int n = 0;
     cudaError_t e = csa::launch_attend(q, q_seq, q_pos, T, H, comp, comp_seq_stride, raw, raw_seq_stride, m, idx, k,

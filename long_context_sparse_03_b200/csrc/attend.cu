@@ -12,14 +12,16 @@
 // 64-row blocks gathered into shared memory with cp.async (the next block is
 // in flight while this one computes), an online softmax in registers, then
 // O += P V with P re-packed from the S accumulators.  The attended row list
-// of a query is cut into fixed 128-row splits (independent of the batch, so
-// results are batch invariant); each CTA writes its split's (max, sum,
-// unnormalised output) and a combine kernel merges the splits in order.
+// of a query is cut into fixed splits (64 rows for CSA, 512 for HCA; never a
+// function of the batch, so results are batch invariant); each CTA writes
+// its split's (max, sum, unnormalised output) and a combine kernel merges
+// the splits in order.
 #include "common.cuh"
 
 namespace csa {
 
-constexpr int kRowsPerSplit = 128;
+constexpr int kCsaRowsPerSplit = 64;    // CSA: k + W rows per query, latency-bound
+constexpr int kHcaRowsPerSplit = 512;   // HCA: thousands of rows per query
 constexpr int kRowBlock = 64;
 constexpr int kRowStride = 136;  // bf16 per smem row (272 B: conflict-free ldmatrix)
 
@@ -37,6 +39,7 @@ struct AttnArgs {
     int max_blocks;  // HCA
     int W;
     float scale_log2;  // scale * log2(e)
+    int rows_per_split;
     int nsplit;
     float* part_o;    // [T][nsplit][H][128]
     float* part_ml;   // [T][nsplit][H][2]
@@ -76,8 +79,8 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
     const int V = a.idx ? (p + 1) / a.m : min((p + 1) / a.m, a.max_blocks);
     const int nsel = a.idx ? a.k : V;
     const int total = nsel + a.W;
-    const int pos0 = sp * kRowsPerSplit;
-    const int npos = max(0, min(kRowsPerSplit, total - pos0));
+    const int pos0 = sp * a.rows_per_split;
+    const int npos = max(0, min(a.rows_per_split, total - pos0));
     const int nblk = (npos + kRowBlock - 1) / kRowBlock;
 
     // issue the gather of row block `blk` into buffer `buf`
@@ -228,30 +231,75 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
     }
 }
 
-// grid (H, T), 128 threads (one per output channel).
+// grid (H, T), 128 threads (one per output channel).  The splits' (max, sum)
+// pairs are staged once in shared memory; each thread then issues all its
+// partial-output loads before combining them in split order.
+constexpr int kCombineMaxSplits = 512;
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                                       int nsplit, int H, bf16* __restrict__ out,
                                                       float* __restrict__ lse) {
+    __shared__ float fac[kCombineMaxSplits];
+    __shared__ float red[2];
     const int h = blockIdx.x, t = blockIdx.y, c = threadIdx.x;
+    // global max over the splits (fixed order reduction: per-thread then warp tree)
     float M = -INFINITY;
-    for (int i = 0; i < nsplit; ++i) M = fmaxf(M, part_ml[(((int64_t)t * nsplit + i) * H + h) * 2]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-        for (int i = 0; i < nsplit; ++i) {
-            const int64_t base = ((int64_t)t * nsplit + i) * H + h;
-            const float mi = part_ml[base * 2];
-            if (mi == -INFINITY) continue;
-            const float f = exp2f(mi - M);
-            L = fmaf(part_ml[base * 2 + 1], f, L);
-            O = fmaf(part_o[base * 128 + c], f, O);
-        }
+    for (int i = c; i < nsplit; i += 128) {
+        const float mi = part_ml[(((int64_t)t * nsplit + i) * H + h) * 2];
+        if (i < kCombineMaxSplits) fac[i] = mi;
+        M = fmaxf(M, mi);
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    __shared__ float wm[4];
+    if ((c & 31) == 0) wm[c >> 5] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+    // per-split factors 2^(m_i - M) (0 for empty splits)
+    for (int i = c; i < nsplit && i < kCombineMaxSplits; i += 128) {
+        const float mi = fac[i];
+        fac[i] = (M == -INFINITY || mi == -INFINITY) ? 0.f : exp2f(mi - M);
+    }
+    __syncthreads();
+    if (c == 0) {
+        float L = 0.f;
+        for (int i = 0; i < nsplit; ++i) {
+            const float f = i < kCombineMaxSplits ? fac[i]
+                                                  : ((M == -INFINITY) ? 0.f
+                                                                      : exp2f(part_ml[(((int64_t)t * nsplit + i) * H + h) * 2] - M));
+            L = fmaf(part_ml[(((int64_t)t * nsplit + i) * H + h) * 2 + 1], f, L);
+        }
+        red[0] = L;
+    }
+    float O = 0.f;
+    int i = 0;
+    for (; i + 4 <= nsplit && i + 4 <= kCombineMaxSplits; i += 4) {   // four loads in flight
+        const float o0 = part_o[(((int64_t)t * nsplit + i) * H + h) * 128 + c];
+        const float o1 = part_o[(((int64_t)t * nsplit + i + 1) * H + h) * 128 + c];
+        const float o2 = part_o[(((int64_t)t * nsplit + i + 2) * H + h) * 128 + c];
+        const float o3 = part_o[(((int64_t)t * nsplit + i + 3) * H + h) * 128 + c];
+        O = fmaf(o0, fac[i], O);
+        O = fmaf(o1, fac[i + 1], O);
+        O = fmaf(o2, fac[i + 2], O);
+        O = fmaf(o3, fac[i + 3], O);
+    }
+    for (; i < nsplit; ++i) {
+        const float f = i < kCombineMaxSplits ? fac[i]
+                                              : ((M == -INFINITY) ? 0.f
+                                                                  : exp2f(part_ml[(((int64_t)t * nsplit + i) * H + h) * 2] - M));
+        O = fmaf(part_o[(((int64_t)t * nsplit + i) * H + h) * 128 + c], f, O);
+    }
+    __syncthreads();
+    const float L = red[0];
     const float res = L > 0.f ? O / L : 0.f;
     out[((int64_t)t * H + h) * 128 + c] = __float2bfloat16_rn(res);
     if (lse && c == 0) lse[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
-int attend_nsplit(int max_rows) { return max_rows <= 0 ? 1 : (max_rows + kRowsPerSplit - 1) / kRowsPerSplit; }
+int attend_rows_per_split(bool dense) { return dense ? kHcaRowsPerSplit : kCsaRowsPerSplit; }
+int attend_nsplit(int max_rows, bool dense) {
+    const int r = attend_rows_per_split(dense);
+    return max_rows <= 0 ? 1 : (max_rows + r - 1) / r;
+}
 
 cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int T, int H, const void* comp,
                           int64_t comp_stride, const void* raw, int64_t raw_stride, int m, const int* idx, int k,
@@ -272,7 +320,8 @@ cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int
     a.W = W;
     a.scale_log2 = scale * 1.4426950408889634f;
     const int max_rows = (idx ? k : max_blocks) + W;
-    a.nsplit = attend_nsplit(max_rows);
+    a.rows_per_split = attend_rows_per_split(idx == nullptr);
+    a.nsplit = attend_nsplit(max_rows, idx == nullptr);
     a.part_o = part_o;
     a.part_ml = part_ml;
     a.status = status;

@@ -6,44 +6,55 @@
 // Readings taken: S_j = sum_h w_h max(0, q_h . k_j) (times the row scale for
 // E4M3 keys); block j visible iff j < (p+1)/m; order = score desc, index asc.
 //
-// Decode is an HBM stream over the compressed indexer keys (64 values per
-// block).  Per key it costs Hi*64 multiply-adds in fp32-grade precision,
-// which at HBM rate is beyond the CUDA-core fp32 rate, so the dot products
-// run on the tensor cores: a warp takes 16 keys as the A operand of
-// mma.m16n8k16 (loaded straight from global memory into registers with
-// 128-bit coalesced loads) and the query heads as the B operand (n = 8 heads
+// Scoring (the HBM stream).  Per key the score costs Hi*64 multiply-adds in
+// fp32-grade precision, beyond the CUDA-core fp32 rate at HBM speed, so the
+// dot products run on the tensor cores: a warp takes 16 keys as the A operand
+// of mma.m16n8k16, loaded straight from global memory into registers with
+// 128-bit coalesced loads, and the query heads as the B operand (n = 8 heads
 // per MMA), split into hi + lo halves so the product keeps ~16 significant
 // bits of q.  The K dimension (the 64 key channels) is permuted so that each
-// lane's fragment is two contiguous 16-byte pieces of a key row; the query
-// fragments use the same permutation, so every dot product is unchanged.
+// lane's fragment is whole 16-byte pieces of a key row; the query fragments
+// use the same permutation, so every dot product is unchanged.  The grid is
+// persistent (a whole number of CTAs per SM): the (query, 256-key unit)
+// pairs are split evenly over the CTAs, a producer warp streams units into a
+// ring of shared-memory stages with TMA bulk copies, and each CTA counts the
+// maximum score of every 32 keys into a 2048-bin histogram of the top 11
+// bits of its order-preserving key.
 //
-// Each CTA keeps its chunk's scores on chip as (score, index) keys, selects
-// its exact local top-k with a shared-memory radix select and writes only
-// those candidates; merge kernels reduce the candidates to the final sorted
-// top-k.  The selection is exact under the total order, so the result does
-// not depend on how the blocks were chunked (batch invariant).
+// Selection.  The k-th largest 32-key maximum is itself a score and has at
+// least k scores at or above it, so it is a lower bound on the k-th largest
+// score; the histogram of tile maxima gives, per query, the bin b* holding
+// it.  A collect pass appends every score at or above that bin's lower edge
+// (about k plus one bin's population) to a candidate list, and a rank pass
+// orders the list exactly: a candidate's slot is the number of candidates
+// above it.
+// Ties are broken by the block index (the candidate key is
+// (score key << 32) | ~index), so the result does not depend on how the
+// work was split: it is batch invariant and deterministic.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace csa {
 
-constexpr int kScoreThreads = 256;
-constexpr int kMergeThreads = 512;
-constexpr int kMergeMax = 16384;  // candidates held by one merge CTA
+constexpr int kUnit = 256;            // keys per work unit (8 warps x 2 tiles of 16)
+constexpr int kHistBins = 2048;       // top 11 bits of the score key
+constexpr int kHistShift = 21;
+constexpr int kCollectKeys = 4096;    // scores scanned per collect CTA
 
 // ---------------------------------------------------------------- select
-// Exact threshold of the kk largest among the distinct nonzero uint64
-// values v[0..n) (zero = empty slot).  Returns thr with exactly
-// min(kk, #nonzero) values >= thr among the nonzero ones (thr = 1 when all
-// are taken).  Every thread of the block must call it.
+// Exact threshold of the kk largest among the distinct nonzero uint64 values
+// v[0..n) (zero = empty).  Returns thr with exactly min(kk, #nonzero) values
+// >= thr among the nonzero ones (thr = 1 when every value is taken).  v may
+// be shared or global memory.  Every thread of the block must call it.
 __device__ uint64_t block_select(const uint64_t* v, int n, int kk, unsigned* hist, int* misc) {
     const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31;
-    // count nonzero
     if (tid == 0) misc[2] = 0;
     __syncthreads();
     int cnt = 0;
     for (int i = tid; i < n; i += nth) cnt += v[i] != 0ull;
     for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (lane == 0) atomicAdd(&misc[2], cnt);
+    if (lane == 0 && cnt) atomicAdd(&misc[2], cnt);
     __syncthreads();
     const int nz = misc[2];
     if (nz <= kk) return 1ull;
@@ -55,7 +66,7 @@ __device__ uint64_t block_select(const uint64_t* v, int n, int kk, unsigned* his
         __syncthreads();
         for (int base = 0; base < n; base += nth) {
             const int i = base + tid;
-            uint64_t x = i < n ? v[i] : 0ull;
+            const uint64_t x = i < n ? v[i] : 0ull;
             const bool match = x != 0ull && (x & mask) == prefix;
             const unsigned dig = (unsigned)(x >> shift) & 255u;
             const unsigned peers = __match_any_sync(0xffffffffu, match ? dig : 0xFFFFFFFFu);
@@ -73,7 +84,7 @@ __device__ uint64_t block_select(const uint64_t* v, int n, int kk, unsigned* his
             unsigned incl = s;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
-                unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+                const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
                 if (lane >= off) incl += o;
             }
             const unsigned excl = incl - s;
@@ -97,14 +108,13 @@ __device__ uint64_t block_select(const uint64_t* v, int n, int kk, unsigned* his
         prefix |= (uint64_t)d << shift;
         mask |= 0xFFull << shift;
         need -= above;
-        __syncthreads();  // misc / hist reused next pass
+        __syncthreads();  // misc / hist are rewritten by the next pass
         if ((int)bin == need) break;
     }
     return prefix;
 }
 
 // ---------------------------------------------------------------- scoring
-// Per-thread query fragments for NT groups of 8 heads.
 template <int NT>
 struct QFrag {
     uint32_t hi[NT][4][2];
@@ -112,10 +122,10 @@ struct QFrag {
     float w[NT][2];
 };
 
-// Physical key channel of (k-step s, lane quarter tq, element e) for bf16
-// keys: lane tq holds 16-byte chunks tq and tq+4 of the 128-byte row.
+// Physical key channel of (k-step s, lane quarter tq, element e): for bf16
+// keys lane tq holds 16-byte chunks tq and tq+4 of the 128-byte row; for
+// E4M3 keys it holds 16-byte chunk tq of the 64-byte row.
 __device__ __forceinline__ int phys_bf16(int s, int tq, int e) { return (s >> 1) * 32 + tq * 8 + (s & 1) * 4 + e; }
-// ... and for E4M3 keys: lane tq holds 16-byte chunk tq of the 64-byte row.
 __device__ __forceinline__ int phys_e4m3(int s, int tq, int e) { return tq * 16 + s * 4 + e; }
 
 template <int FMT, int NT>
@@ -160,39 +170,44 @@ __device__ void load_qfrag(QFrag<NT>& f, const float* q_sh, const float* w_sh, c
     }
 }
 
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
 // Raw key bytes of one 16-key tile for this lane.
 struct KeyTile {
     uint4 a0, a1, b0, b1;  // bf16: rows g, g+8, chunks tq / tq+4; E4M3: a0, a1 only
     float s0, s1;          // E4M3 row scales
 };
 
+// Read the lane's part of the tile whose first row is `row0` of a stage.
+// bf16 rows are 128 B: odd rows read their two chunks in the other order so
+// that each quarter-warp touches 32 distinct banks.
 template <int FMT>
-__device__ __forceinline__ void load_tile(KeyTile& kt, const uint8_t* kbase, const float* sbase, int r0, int j1) {
+__device__ __forceinline__ void smem_tile(KeyTile& kt, const uint8_t* stage, int row0) {
     const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int ra = r0 + g, rb = r0 + g + 8;
-    const uint4 z = make_uint4(0, 0, 0, 0);
     if (FMT == 0) {
-        const uint8_t* pa = kbase + (int64_t)ra * 128 + tq * 16;
-        const uint8_t* pb = kbase + (int64_t)rb * 128 + tq * 16;
-        kt.a0 = ra < j1 ? ldg_stream(pa) : z;
-        kt.b0 = ra < j1 ? ldg_stream(pa + 64) : z;
-        kt.a1 = rb < j1 ? ldg_stream(pb) : z;
-        kt.b1 = rb < j1 ? ldg_stream(pb + 64) : z;
+        const bool odd = g & 1;
+        const uint8_t* ra = stage + (row0 + g) * 128;
+        const uint8_t* rb = ra + 8 * 128;
+        const int c1 = odd ? tq + 4 : tq, c2 = odd ? tq : tq + 4;
+        const uint4 x0 = *reinterpret_cast<const uint4*>(ra + c1 * 16);
+        const uint4 x1 = *reinterpret_cast<const uint4*>(ra + c2 * 16);
+        const uint4 y0 = *reinterpret_cast<const uint4*>(rb + c1 * 16);
+        const uint4 y1 = *reinterpret_cast<const uint4*>(rb + c2 * 16);
+        kt.a0 = odd ? x1 : x0;
+        kt.b0 = odd ? x0 : x1;
+        kt.a1 = odd ? y1 : y0;
+        kt.b1 = odd ? y0 : y1;
     } else {
-        kt.a0 = ra < j1 ? ldg_stream(kbase + (int64_t)ra * 64 + tq * 16) : z;
-        kt.a1 = rb < j1 ? ldg_stream(kbase + (int64_t)rb * 64 + tq * 16) : z;
-        kt.s0 = ra < j1 ? __ldg(sbase + ra) : 0.f;
-        kt.s1 = rb < j1 ? __ldg(sbase + rb) : 0.f;
+        kt.a0 = *reinterpret_cast<const uint4*>(stage + (row0 + g) * 64 + tq * 16);
+        kt.a1 = *reinterpret_cast<const uint4*>(stage + (row0 + g + 8) * 64 + tq * 16);
     }
 }
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xFFFFu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
-// Scores of the lane's two rows (g, g+8) of one tile (valid in every lane
-// of the quad after the reduction).
+// Scores of the lane's two rows (g, g+8) of one tile (the same in all four
+// lanes of the quad after the reduction).
 template <int FMT, int NT>
 __device__ __forceinline__ void score_tile(const KeyTile& kt, const QFrag<NT>& f, float& s0, float& s1) {
     float c[NT][4];
@@ -248,275 +263,589 @@ __device__ __forceinline__ void score_tile(const KeyTile& kt, const QFrag<NT>& f
     s1 = p1;
 }
 
-// grid (nchunks, T), 256 threads.  MODE 0: write exact local top-kc
-// candidates of the chunk to cand[t][chunk][kc].  MODE 1: write the raw
-// scores to scores[t][max_blocks] (NaN past V(t)).
-template <int FMT, int NT, int MODE>
-__global__ void __launch_bounds__(kScoreThreads, 2) index_score_kernel(
-    const float* __restrict__ q, const float* __restrict__ w, const int* __restrict__ q_seq,
-    const int* __restrict__ q_pos, int Hi, const uint8_t* __restrict__ kidx,
-    const float* __restrict__ kscale, int64_t kstride_bytes, int64_t sstride, int m, int max_blocks,
-    int chunk, int kc, uint64_t* __restrict__ cand, float* __restrict__ scores) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint64_t* cand_sh = reinterpret_cast<uint64_t*>(smem_raw);             // [chunk]
-    float* q_sh = reinterpret_cast<float*>(smem_raw + (size_t)chunk * 8);  // [16*64]
-    float* w_sh = q_sh + 16 * 64;                                          // [16]
-    int* e_sh = reinterpret_cast<int*>(w_sh + 16);                         // [16]
-    unsigned* hist = reinterpret_cast<unsigned*>(e_sh + 16);               // [256]
-    int* misc = reinterpret_cast<int*>(hist + 256);                        // [4]
-
-    const int t = blockIdx.y, ch = blockIdx.x;
-    const int b = q_seq[t];
-    const int V = min((q_pos[t] + 1) / m, max_blocks);
-    const int j0 = ch * chunk;
-    const int j1 = min(j0 + chunk, V);
-    const int n = max(0, j1 - j0);
-
-    if (MODE == 1) {
-        for (int j = max(j0, V) + threadIdx.x; j < min(j0 + chunk, max_blocks); j += blockDim.x)
-            scores[(int64_t)t * max_blocks + j] = __int_as_float(0x7fc00000);
+// Two tiles at once (independent accumulators: twice the MMA chains in
+// flight per warp).
+template <int FMT, int NT>
+__device__ __forceinline__ void score_tile2(const KeyTile* kt, const QFrag<NT>& f, float (*sc)[2]) {
+    float c[2][NT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) c[h][nt][0] = c[h][nt][1] = c[h][nt][2] = c[h][nt][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t a[4];
+            if (FMT == 0) {
+                const uint4& A = (s < 2) ? kt[h].a0 : kt[h].b0;
+                const uint4& Bq = (s < 2) ? kt[h].a1 : kt[h].b1;
+                const bool hiw = s & 1;
+                a[0] = hiw ? A.z : A.x;
+                a[2] = hiw ? A.w : A.y;
+                a[1] = hiw ? Bq.z : Bq.x;
+                a[3] = hiw ? Bq.w : Bq.y;
+            } else {
+                const uint4& A = kt[h].a0;
+                const uint4& Bq = kt[h].a1;
+                const uint32_t wa = s == 0 ? A.x : s == 1 ? A.y : s == 2 ? A.z : A.w;
+                const uint32_t wb = s == 0 ? Bq.x : s == 1 ? Bq.y : s == 2 ? Bq.z : Bq.w;
+                a[0] = e4m3x2_to_f16x2(wa);
+                a[2] = e4m3x2_to_f16x2(wa >> 16);
+                a[1] = e4m3x2_to_f16x2(wb);
+                a[3] = e4m3x2_to_f16x2(wb >> 16);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                if (FMT == 0) {
+                    mma_bf16_16816(c[h][nt], a, f.hi[nt][s][0], f.hi[nt][s][1]);
+                    mma_bf16_16816(c[h][nt], a, f.lo[nt][s][0], f.lo[nt][s][1]);
+                } else {
+                    mma_f16_16816(c[h][nt], a, f.hi[nt][s][0], f.hi[nt][s][1]);
+                    mma_f16_16816(c[h][nt], a, f.lo[nt][s][0], f.lo[nt][s][1]);
+                }
+            }
+        }
     }
-    if (n == 0) {
-        if (MODE == 0)
-            for (int i = threadIdx.x; i < kc; i += blockDim.x) cand[((int64_t)t * gridDim.x + ch) * kc + i] = 0ull;
-        return;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            p0 = fmaf(f.w[nt][0], fmaxf(c[h][nt][0], 0.f), p0);
+            p0 = fmaf(f.w[nt][1], fmaxf(c[h][nt][1], 0.f), p0);
+            p1 = fmaf(f.w[nt][0], fmaxf(c[h][nt][2], 0.f), p1);
+            p1 = fmaf(f.w[nt][1], fmaxf(c[h][nt][3], 0.f), p1);
+        }
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+        p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+        p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+        if (FMT == 1) {
+            p0 *= kt[h].s0;
+            p1 *= kt[h].s1;
+        }
+        sc[h][0] = p0;
+        sc[h][1] = p1;
     }
+}
 
-    for (int i = threadIdx.x; i < Hi * 64; i += blockDim.x) q_sh[i] = q[(int64_t)t * Hi * 64 + i];
-    if (threadIdx.x < Hi) w_sh[threadIdx.x] = w[(int64_t)t * Hi + threadIdx.x];
-    __syncthreads();
-    if (FMT == 1 && threadIdx.x < Hi) {
+struct ScoreArgs {
+    const float* q;       // [T][Hi][64]
+    const float* w;       // [T][Hi]
+    const int* q_seq;
+    const int* q_pos;
+    int T, Hi, m, max_blocks, k;
+    const uint8_t* kidx;
+    const float* kscale;
+    int64_t kstride_bytes, sstride;
+    float* scores;        // [T][ld_scores]
+    int64_t ld_scores;
+    unsigned* hist;       // [T][kHistBins] or nullptr (scores only)
+    unsigned* done;       // [T] CTAs finished per query
+    unsigned* thr;        // [T] threshold key per query (written by the last CTA)
+    unsigned* status;     // device status word (timeouts)
+    int units_per_q;      // ceil(max_blocks / kUnit)
+};
+
+constexpr int kConsumers = 256;                   // 8 consumer warps
+constexpr int kScoreCta = kConsumers + 32;        // + 1 producer warp
+constexpr unsigned kWaitTries = 1u << 22;         // bounded mbarrier waits
+
+template <int FMT>
+struct ScoreCfg;
+template <>
+struct ScoreCfg<0> {
+    static constexpr int kRow = 128;      // bytes per key row
+    static constexpr int kStages = 3;     // 3 x 32 KB in flight per CTA
+};
+template <>
+struct ScoreCfg<1> {
+    static constexpr int kRow = 64;
+    static constexpr int kStages = 6;     // 6 x 16 KB
+};
+
+struct ScoreSmem {
+    float q_sh[16 * 64];
+    float w_sh[16];
+    int e_sh[16];
+    unsigned hsh[kHistBins];
+    unsigned scan_sh[kConsumers];
+    int misc[4];
+};
+
+template <int FMT>
+constexpr size_t score_smem_bytes() {
+    return (size_t)ScoreCfg<FMT>::kStages * kUnit * ScoreCfg<FMT>::kRow + 2 * 8 * ScoreCfg<FMT>::kStages +
+           sizeof(ScoreSmem);
+}
+
+// Per-query fragments (q, w staged through shared memory); consumers only.
+template <int FMT, int NT>
+__device__ void enter_query(const ScoreArgs& a, int t, QFrag<NT>& f, ScoreSmem& sm) {
+    named_sync(1, kConsumers);
+    for (int i = threadIdx.x; i < a.Hi * 64; i += kConsumers) sm.q_sh[i] = a.q[(int64_t)t * a.Hi * 64 + i];
+    if (threadIdx.x < a.Hi) sm.w_sh[threadIdx.x] = a.w[(int64_t)t * a.Hi + threadIdx.x];
+    named_sync(1, kConsumers);
+    if (FMT == 1 && threadIdx.x < a.Hi) {
         // power-of-two scale per head so its largest |q| sits in [2^14, 2^15)
         float amax = 0.f;
-        for (int c = 0; c < 64; ++c) amax = fmaxf(amax, fabsf(q_sh[threadIdx.x * 64 + c]));
+        for (int c = 0; c < 64; ++c) amax = fmaxf(amax, fabsf(sm.q_sh[threadIdx.x * 64 + c]));
         int ex = 0;
         if (amax > 0.f) {
             int e2;
             frexpf(amax, &e2);
             ex = 15 - e2;
         }
-        e_sh[threadIdx.x] = ex;
+        sm.e_sh[threadIdx.x] = ex;
     }
-    __syncthreads();
+    named_sync(1, kConsumers);
+    load_qfrag<FMT, NT>(f, sm.q_sh, sm.w_sh, sm.e_sh, a.Hi);
+}
 
-    QFrag<NT> f;
-    load_qfrag<FMT, NT>(f, q_sh, w_sh, e_sh, Hi);
-
-    const uint8_t* kbase = kidx + (int64_t)b * kstride_bytes;
-    const float* sbase = FMT == 1 ? kscale + (int64_t)b * sstride : nullptr;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int ntiles = (n + 15) >> 4;
-
-    // two tiles per step, the next pair prefetched while this one computes
-    KeyTile cur[2], nxt[2];
-    int tile = warp;
+// Highest bin b with (#counts in bins >= b) >= k (0 when fewer than k):
+// the k-th largest counted tile maximum lies in bin b, so b's lower edge is
+// a lower bound on the k-th largest score.
+// Consumers only (256 threads, 16 bins each).
+__device__ unsigned threshold_bin(const unsigned* ghist, int k, unsigned* sh, int* misc) {
+    const int tid = threadIdx.x;
+    constexpr int per = kHistBins / kConsumers;
+    unsigned c[per], s = 0;
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
-        if (tile + 8 * u < ntiles) load_tile<FMT>(cur[u], kbase, sbase, j0 + (tile + 8 * u) * 16, j1);
-    for (; tile < ntiles; tile += 16) {
+    for (int e = 0; e < per; ++e) {
+        c[e] = __ldcg(&ghist[kHistBins - 1 - (tid * per + e)]);
+        s += c[e];
+    }
+    sh[tid] = s;
+    if (tid == 0) misc[0] = 0;
+    named_sync(1, kConsumers);
+    for (int off = 1; off < kConsumers; off <<= 1) {   // inclusive scan, top bins first
+        const unsigned v = tid >= off ? sh[tid - off] : 0u;
+        named_sync(1, kConsumers);
+        sh[tid] += v;
+        named_sync(1, kConsumers);
+    }
+    const unsigned incl = sh[tid], excl = incl - s;
+    if (excl < (unsigned)k && (unsigned)k <= incl) {
+        unsigned run = excl;
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-            if (tile + 16 + 8 * u < ntiles) load_tile<FMT>(nxt[u], kbase, sbase, j0 + (tile + 16 + 8 * u) * 16, j1);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int tl = tile + 8 * u;
-            if (tl < ntiles) {
-                float s0, s1;
-                score_tile<FMT, NT>(cur[u], f, s0, s1);
-                const int ra = j0 + tl * 16 + g, rb = ra + 8;
-                if (tq == 0) {
-                    if (MODE == 0) {
-                        if (ra < j1) cand_sh[ra - j0] = make_cand(s0, ra);
-                        if (rb < j1) cand_sh[rb - j0] = make_cand(s1, rb);
-                    } else {
-                        if (ra < j1) scores[(int64_t)t * max_blocks + ra] = s0;
-                        if (rb < j1) scores[(int64_t)t * max_blocks + rb] = s1;
-                    }
-                }
+        for (int e = 0; e < per; ++e) {
+            run += c[e];
+            if (run >= (unsigned)k) {
+                misc[0] = kHistBins - 1 - (tid * per + e);
+                break;
             }
         }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) cur[u] = nxt[u];
     }
-    if (MODE == 1) return;
-    __syncthreads();
+    named_sync(1, kConsumers);
+    const unsigned b = (unsigned)misc[0];
+    named_sync(1, kConsumers);
+    return b;
+}
 
-    uint64_t* dst = cand + ((int64_t)t * gridDim.x + ch) * kc;
-    if (n <= kc) {
-        for (int i = threadIdx.x; i < kc; i += blockDim.x) dst[i] = i < n ? cand_sh[i] : 0ull;
-        return;
+// Leave query t: add the CTA's shared histogram to the query's global one;
+// the CTA that completes the query turns it into the threshold key.
+__device__ void leave_query(const ScoreArgs& a, int t, int contributors, ScoreSmem& sm) {
+    named_sync(1, kConsumers);
+    unsigned* gh = a.hist + (int64_t)t * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += kConsumers) {
+        const unsigned c = sm.hsh[i];
+        if (c) {
+            atomicAdd(&gh[i], c);
+            sm.hsh[i] = 0;
+        }
     }
-    const uint64_t thr = block_select(cand_sh, n, kc, hist, misc);
-    if (threadIdx.x == 0) misc[3] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint64_t x = cand_sh[i];
-        if (x >= thr) dst[atomicAdd(&misc[3], 1)] = x;
+    __threadfence();
+    named_sync(1, kConsumers);
+    if (threadIdx.x == 0) sm.misc[1] = atomicAdd(&a.done[t], 1u) == (unsigned)(contributors - 1);
+    named_sync(1, kConsumers);
+    if (sm.misc[1]) {
+        __threadfence();
+        const unsigned b = threshold_bin(gh, a.k, sm.scan_sh, sm.misc);
+        if (threadIdx.x == 0) a.thr[t] = b << kHistShift;
     }
 }
 
-// ---------------------------------------------------------------- merge
-// grid (ngroups, T).  CTA takes candidates [g*group, min((g+1)*group, n)) of
-// query t.  FINAL: sort the top-k (score desc, index asc) and write
-// out_idx / out_score; else write k candidates to out[t][g][k].
-template <bool FINAL>
-__global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint64_t* __restrict__ in, int n, int group,
-                                                              int k, uint64_t* __restrict__ out,
-                                                              int* __restrict__ out_idx,
-                                                              float* __restrict__ out_score) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    uint64_t* v = reinterpret_cast<uint64_t*>(smem_raw);  // [group]
-    unsigned* hist = reinterpret_cast<unsigned*>(v + group);
-    int* misc = reinterpret_cast<int*>(hist + 256);
-    uint64_t* srt = reinterpret_cast<uint64_t*>(misc + 8);  // [P] (FINAL)
+// CTA that owns work unit x under the even split of U units over G CTAs.
+__device__ __forceinline__ int owner_cta(int64_t x, int64_t U, int64_t G) { return (int)(((x + 1) * G - 1) / U); }
 
-    const int t = blockIdx.y, gi = blockIdx.x;
-    const int lo = gi * group, cnt = min(group, n - lo);
-    const uint64_t* src = in + (int64_t)t * n + lo;
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) v[i] = src[i];
-    __syncthreads();
-    const uint64_t thr = block_select(v, cnt, k, hist, misc);
+// Persistent, warp-specialised scoring kernel.  CTA c takes work units
+// [u_lo, u_hi) of the flattened (query, 128-key unit) space.  Warp 8 is the
+// producer: one lane streams each unit's key rows into a ring of shared
+// memory stages with 1-D TMA bulk copies (completion counted on a "full"
+// mbarrier per stage).  Warps 0-7 consume: each scores two 16-key tiles of
+// the unit on the tensor cores, then releases the stage on its "empty"
+// barrier.
+// Every wait is bounded; a wait that runs out flags CSA_DEV_TIMEOUT and the
+// CTA carries on (treating the unit as empty), so it always exits.
+template <int FMT, int NT>
+__global__ void __launch_bounds__(kScoreCta, 2) index_score_kernel(ScoreArgs a) {
+    constexpr int S = ScoreCfg<FMT>::kStages;
+    constexpr int ROW = ScoreCfg<FMT>::kRow;
+    constexpr int UNIT_BYTES = kUnit * ROW;
+    extern __shared__ __align__(128) uint8_t smem_score[];
+    uint8_t* stages = smem_score;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem_score + (size_t)S * UNIT_BYTES);
+    uint64_t* empty = full + S;
+    ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(empty + S);
 
-    if (!FINAL) {
-        uint64_t* dst = out + ((int64_t)t * gridDim.x + gi) * k;
-        if (threadIdx.x == 0) misc[3] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-            const uint64_t x = v[i];
-            if (x != 0ull && x >= thr) dst[atomicAdd(&misc[3], 1)] = x;
+    const int64_t U = (int64_t)a.T * a.units_per_q, G = gridDim.x;
+    const int64_t u_lo = U * blockIdx.x / G, u_hi = U * (blockIdx.x + 1) / G;
+    if (u_lo >= u_hi) return;
+    const int64_t n_units = u_hi - u_lo;
+    const int upq = a.units_per_q;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumers / 32);
         }
-        __syncthreads();
-        for (int i = misc[3] + threadIdx.x; i < k; i += blockDim.x) dst[i] = 0ull;
-        return;
+        fence_mbar_init();
     }
-    int P = 1;
-    while (P < k) P <<= 1;
-    for (int i = threadIdx.x; i < P; i += blockDim.x) srt[i] = 0ull;
-    if (threadIdx.x == 0) misc[3] = 0;
+    for (int i = threadIdx.x; i < kHistBins; i += kScoreCta) sm.hsh[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-        const uint64_t x = v[i];
-        if (x != 0ull && x >= thr) srt[atomicAdd(&misc[3], 1)] = x;
-    }
-    __syncthreads();
-    // bitonic sort, descending
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
-                const int pos = 2 * i - (i & (stride - 1));
-                const int par = pos + stride;
-                const bool desc = (pos & size) == 0;
-                const uint64_t x = srt[pos], y = srt[par];
-                if ((x < y) == desc) {
-                    srt[pos] = y;
-                    srt[par] = x;
+
+    auto vis = [&](int t) { return min((a.q_pos[t] + 1) / a.m, a.max_blocks); };
+
+    if (warp == kConsumers / 32) {
+        // ------------------------------------------------ producer warp
+        if (lane == 0) {
+            int pt = (int)(u_lo / upq), pub = (int)(u_lo % upq);
+            int pV = vis(pt);
+            const uint8_t* pkb = a.kidx + (int64_t)a.q_seq[pt] * a.kstride_bytes;
+            int slot = 0;
+            unsigned phase = 0;
+            for (int64_t i = 0; i < n_units; ++i) {
+                if (i >= S && !mbar_wait_bounded(&empty[slot], phase ^ 1u, kWaitTries))
+                    flag_status(a.status, kDevTimeout);
+                const int rows = max(0, min(kUnit, pV - pub * kUnit));
+                if (rows > 0) {
+                    mbar_arrive_expect_tx(&full[slot], (unsigned)(rows * ROW));
+                    bulk_g2s(stages + (size_t)slot * UNIT_BYTES, pkb + (int64_t)pub * UNIT_BYTES,
+                             (unsigned)(rows * ROW), &full[slot]);
+                } else {
+                    mbar_arrive(&full[slot]);
+                }
+                if (++pub == upq) {
+                    pub = 0;
+                    if (++pt < a.T) {
+                        pV = vis(pt);
+                        pkb = a.kidx + (int64_t)a.q_seq[pt] * a.kstride_bytes;
+                    }
+                }
+                if (++slot == S) {
+                    slot = 0;
+                    phase ^= 1u;
                 }
             }
-            __syncthreads();
+            // drain: the last phase of every stage has landed before exit
+            for (int s = 0; s < S && s < n_units; ++s) {
+                const int64_t last = s + ((n_units - 1 - s) / S) * S;
+                if (!mbar_wait_bounded(&full[s], (unsigned)(last / S) & 1u, kWaitTries))
+                    flag_status(a.status, kDevTimeout);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------- consumer warps
+    const int g = lane >> 2, tq = lane & 3;
+    auto contrib = [&](int t) {
+        return owner_cta((int64_t)(t + 1) * upq - 1, U, G) - owner_cta((int64_t)t * upq, U, G) + 1;
+    };
+    int ct = (int)(u_lo / upq), cub = (int)(u_lo % upq), V = 0;
+    bool fresh = true;
+    float* srow = nullptr;
+    const float* sbase = nullptr;
+    QFrag<NT> f;
+    int slot = 0;
+    unsigned phase = 0;
+    for (int64_t i = 0; i < n_units; ++i) {
+        if (i > 0 && ++cub == upq) {   // uniform across the consumers
+            if (a.hist) leave_query(a, ct, contrib(ct), sm);
+            cub = 0;
+            ++ct;
+            fresh = true;
+        }
+        if (fresh) {
+            fresh = false;
+            V = vis(ct);
+            srow = a.scores + (int64_t)ct * a.ld_scores;
+            if (FMT == 1) sbase = a.kscale + (int64_t)a.q_seq[ct] * a.sstride;
+            enter_query<FMT, NT>(a, ct, f, sm);
+        }
+        const int r0 = cub * kUnit + warp * 32;   // first block index of the warp's two tiles
+        KeyTile kt[2];
+        if (FMT == 1) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int ra = r0 + 16 * h + g, rb = ra + 8;
+                kt[h].s0 = ra < V ? __ldg(sbase + ra) : 0.f;
+                kt[h].s1 = rb < V ? __ldg(sbase + rb) : 0.f;
+            }
+        }
+        const bool landed = mbar_wait_bounded(&full[slot], phase, kWaitTries);
+        if (!landed && lane == 0) flag_status(a.status, kDevTimeout);
+        if (landed && r0 < V) {   // uniform across the warp
+            // rows past V inside a tile hold stale bytes: their scores are dropped
+            const uint8_t* st = stages + (size_t)slot * UNIT_BYTES;
+            smem_tile<FMT>(kt[0], st, warp * 32);
+            smem_tile<FMT>(kt[1], st, warp * 32 + 16);
+            float sc[2][2];
+            score_tile2<FMT, NT>(kt, f, sc);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int ra = r0 + 16 * h + g, rb = ra + 8;
+                if (tq == 0) {
+                    if (ra < V) srow[ra] = sc[h][0];
+                    if (rb < V) srow[rb] = sc[h][1];
+                }
+                mx = fmaxf(mx, fmaxf(ra < V ? sc[h][0] : -INFINITY, rb < V ? sc[h][1] : -INFINITY));
+            }
+            if (a.hist) {
+                // histogram of the maximum of the warp's 32 keys
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                if (lane == 0) atomicAdd(&sm.hsh[score_key(mx) >> kHistShift], 1u);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (++slot == S) {
+            slot = 0;
+            phase ^= 1u;
         }
     }
-    const int nsel = misc[3];
-    for (int i = threadIdx.x; i < k; i += blockDim.x) {
-        const uint64_t x = srt[i];
-        const bool ok = i < nsel;
-        out_idx[(int64_t)t * k + i] = ok ? cand_index(x) : -1;
-        if (out_score) out_score[(int64_t)t * k + i] = ok ? cand_score(x) : __int_as_float(0x7fc00000);
+    if (a.hist) leave_query(a, ct, contrib(ct), sm);
+}
+
+// ---------------------------------------------------------------- collect
+// grid (ceil(max_blocks / kCollectKeys), T), 256 threads: append every score
+// whose key reaches the query's threshold to its candidate list.
+__global__ void __launch_bounds__(256) collect_kernel(const float* __restrict__ scores, int64_t ld_scores,
+                                                      const unsigned* __restrict__ thr_t, const int* __restrict__ q_pos,
+                                                      int m, int max_blocks, uint64_t* __restrict__ cand,
+                                                      int64_t cand_cap, unsigned* __restrict__ cnt) {
+    const int t = blockIdx.y;
+    const int V = min((q_pos[t] + 1) / m, max_blocks);
+    const int j0 = blockIdx.x * kCollectKeys;
+    if (j0 >= V) return;
+    const uint32_t thr = thr_t[t];
+    const float* srow = scores + (int64_t)t * ld_scores;
+    uint64_t* crow = cand + (int64_t)t * cand_cap;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int j1 = min(j0 + kCollectKeys, V);
+    constexpr int PER = kCollectKeys / 256;
+    __shared__ unsigned wcount[8], wbase[8];
+    float sv[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {   // all loads in flight before any use
+        const int j = j0 + e * 256 + threadIdx.x;
+        sv[e] = j < j1 ? srow[j] : 0.f;
+    }
+    unsigned bal[PER], mine = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        const int j = j0 + e * 256 + threadIdx.x;
+        bal[e] = __ballot_sync(0xffffffffu, j < j1 && score_key(sv[e]) >= thr);
+        mine += __popc(bal[e]);
+    }
+    if (lane == 0) wcount[warp] = mine;
+    __syncthreads();
+    if (threadIdx.x == 0) {   // one atomic per CTA
+        unsigned tot = 0;
+        for (int w = 0; w < 8; ++w) {
+            wbase[w] = tot;
+            tot += wcount[w];
+        }
+        const unsigned base = tot ? atomicAdd(&cnt[t], tot) : 0u;
+        for (int w = 0; w < 8; ++w) wbase[w] += base;
+    }
+    __syncthreads();
+    unsigned pos = wbase[warp];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        if (bal[e] >> lane & 1u) {
+            const int j = j0 + e * 256 + threadIdx.x;
+            crow[pos + __popc(bal[e] & ((1u << lane) - 1u))] = make_cand(sv[e], j);
+        }
+        pos += __popc(bal[e]);
+    }
+}
+
+// ---------------------------------------------------------------- final
+// Exact selection and ordering of a query's candidate list (n ~ k plus one
+// histogram bin).  grid (kRankCtas, T), kRankThreads threads.  Every CTA
+// stages the whole list in shared memory, finds the exact k-th largest key
+// with a radix select, compacts the k selected keys, and ranks its share of
+// them: a selected key's output slot is the number of selected keys above it
+// (all keys are distinct).  Lists longer than kRankCap are selected from
+// global memory by CTA 0 alone.
+constexpr int kRankThreads = 256;
+constexpr int kRankCtas = 16;
+constexpr int kRankCap = 12288;       // candidates held in shared memory (96 KB)
+constexpr int kRankSplit = 4;         // threads per ranked key
+
+__device__ __forceinline__ void write_out(int* out_idx, float* out_score, int64_t pos, uint64_t x) {
+    out_idx[pos] = cand_index(x);
+    if (out_score) out_score[pos] = cand_score(x);
+}
+
+__global__ void __launch_bounds__(kRankThreads) rank_kernel(const uint64_t* __restrict__ cand, int64_t cand_cap,
+                                                          const unsigned* __restrict__ cnt, int k,
+                                                          int* __restrict__ out_idx, float* __restrict__ out_score) {
+    extern __shared__ __align__(16) uint64_t v[];   // [kRankCap] list, then [CSA k max] selected
+    __shared__ unsigned hist[256];
+    __shared__ int misc[8];
+    uint64_t* sel = v + kRankCap;
+    const int t = blockIdx.y, r = blockIdx.x;
+    const int n = (int)cnt[t];
+    const uint64_t* src = cand + (int64_t)t * cand_cap;
+    if (r == 0)   // padding when fewer than k candidates exist
+        for (int i = n + threadIdx.x; i < k; i += blockDim.x) {
+            out_idx[(int64_t)t * k + i] = -1;
+            if (out_score) out_score[(int64_t)t * k + i] = __int_as_float(0x7fc00000);
+        }
+    const bool in_smem = n <= kRankCap;
+    if (!in_smem && r != 0) return;
+    if (in_smem) {
+        // stage with cp.async (every 16-byte piece in flight); an odd last
+        // element is zero-filled past the end
+        for (int i = 2 * threadIdx.x; i < n; i += 2 * blockDim.x) cp_async16(v + i, src + i, i + 1 < n ? 16 : 8);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+    }
+    const uint64_t* list = in_smem ? v : src;
+    const uint64_t thr = block_select(list, n, k, hist, misc);
+    // order-preserving compaction: every CTA builds the same array
+    __shared__ unsigned wcnt[kRankThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int ns = 0;
+    for (int base = 0; base < n; base += kRankThreads) {
+        const int i = base + threadIdx.x;
+        const uint64_t x = i < n ? list[i] : 0ull;
+        const bool take = x != 0ull && x >= thr;
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) wcnt[warp] = __popc(bal);
+        __syncthreads();
+        int off = ns, tot = 0;
+        for (int w2 = 0; w2 < kRankThreads / 32; ++w2) {
+            if (w2 < warp) off += wcnt[w2];
+            tot += wcnt[w2];
+        }
+        if (take) sel[off + __popc(bal & ((1u << lane) - 1u))] = x;
+        ns += tot;
+        __syncthreads();
+    }
+    // ns = min(k, n)
+    // this CTA's share of the selected keys (all of them when the list was long)
+    const int c0 = in_smem ? (int)((int64_t)ns * r / kRankCtas) : 0;
+    const int c1 = in_smem ? (int)((int64_t)ns * (r + 1) / kRankCtas) : ns;
+    for (int base = c0; base < c1; base += kRankThreads / kRankSplit) {
+        const int e = base + threadIdx.x / kRankSplit, part = threadIdx.x % kRankSplit;
+        const uint64_t x = e < c1 ? sel[e] : ~0ull;
+        int r0 = 0, r1 = 0;
+        int j = part;
+        for (; j + kRankSplit < ns; j += 2 * kRankSplit) {
+            r0 += sel[j] > x;
+            r1 += sel[j + kRankSplit] > x;
+        }
+        if (j < ns) r0 += sel[j] > x;
+        int rank = r0 + r1;
+#pragma unroll
+        for (int off = 1; off < kRankSplit; off <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, off);
+        if (part == 0 && e < c1) write_out(out_idx, out_score, (int64_t)t * k + rank, x);
     }
 }
 
 // ---------------------------------------------------------------- host
-int score_chunk(int T, int max_blocks) {
-    for (int c = 8192; c > 1024; c >>= 1)
-        if ((int64_t)T * ((max_blocks + c - 1) / c) >= 512) return c;
-    return 1024;
-}
+static int g_sm_count[64];
+static int g_score_occ[64][2][2];
 
-struct SelectPlan {
-    int chunk, nchunks, kc;
-    int64_t n0;              // candidates per query after scoring
-    size_t cand_a, cand_b;   // bytes of the two candidate buffers
-};
-
-SelectPlan plan_select(int T, int max_blocks, int k) {
-    SelectPlan p;
-    p.chunk = score_chunk(T, max_blocks);
-    p.nchunks = (max_blocks + p.chunk - 1) / p.chunk;
-    if (p.nchunks < 1) p.nchunks = 1;
-    p.kc = k < p.chunk ? k : p.chunk;
-    p.n0 = (int64_t)p.nchunks * p.kc;
-    p.cand_a = (size_t)T * (size_t)p.n0 * 8;
-    int64_t n = p.n0, maxb = 0;
-    while (n > kMergeMax) {
-        const int64_t ng = (n + kMergeMax - 1) / kMergeMax;
-        n = ng * k;
-        if (n > maxb) maxb = n;
+static int sm_count(int dev) {
+    if (dev < 0 || dev >= 64) return 148;
+    if (!g_sm_count[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        g_sm_count[dev] = n;
     }
-    p.cand_b = (size_t)T * (size_t)maxb * 8;
-    return p;
+    return g_sm_count[dev];
 }
 
-static size_t score_smem(int chunk) { return (size_t)chunk * 8 + 16 * 64 * 4 + 16 * 4 + 16 * 4 + 256 * 4 + 16; }
-
-cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
-                               const void* kidx, int fmt, const float* kscale, int64_t kstride_elems,
-                               int64_t sstride, int m, int max_blocks, int k, uint64_t* cand, float* scores,
-                               cudaStream_t stream, int* launches) {
-    const SelectPlan p = plan_select(T, max_blocks, k);
-    const int chunk = p.chunk;
-    dim3 grid(p.nchunks, T);
-    const size_t smem = score_smem(chunk);
-    const int64_t kbytes = kstride_elems * (fmt == 0 ? 2 : 1);
-    const uint8_t* kb = reinterpret_cast<const uint8_t*>(kidx);
-    const bool dbg = scores != nullptr;
-    const int nt = Hi > 8 ? 2 : 1;
-#define CSA_LAUNCH_SCORE(F, N, MD)                                                                      \
-    do {                                                                                                \
-        auto kern = index_score_kernel<F, N, MD>;                                                       \
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-        if (e != cudaSuccess) return e;                                                                 \
-        kern<<<grid, kScoreThreads, smem, stream>>>(q, w, q_seq, q_pos, Hi, kb, kscale, kbytes, sstride, m, \
-                                                    max_blocks, chunk, p.kc, cand, scores);             \
-    } while (0)
-    if (fmt == 0) {
-        if (nt == 1) { if (dbg) CSA_LAUNCH_SCORE(0, 1, 1); else CSA_LAUNCH_SCORE(0, 1, 0); }
-        else         { if (dbg) CSA_LAUNCH_SCORE(0, 2, 1); else CSA_LAUNCH_SCORE(0, 2, 0); }
-    } else {
-        if (nt == 1) { if (dbg) CSA_LAUNCH_SCORE(1, 1, 1); else CSA_LAUNCH_SCORE(1, 1, 0); }
-        else         { if (dbg) CSA_LAUNCH_SCORE(1, 2, 1); else CSA_LAUNCH_SCORE(1, 2, 0); }
-    }
-#undef CSA_LAUNCH_SCORE
-    *launches += 1;
-    return cudaGetLastError();
-}
-
-cudaError_t launch_index_merge(int T, int max_blocks, int k, uint64_t* cand_a, uint64_t* cand_b, int* out_idx,
-                               float* out_score, cudaStream_t stream, int* launches) {
-    const SelectPlan p = plan_select(T, max_blocks, k);
-    int64_t n = p.n0;
-    uint64_t* src = cand_a;
-    uint64_t* dst = cand_b;
-    while (n > kMergeMax) {
-        const int ng = (int)((n + kMergeMax - 1) / kMergeMax);
-        const size_t smem = (size_t)kMergeMax * 8 + 256 * 4 + 32;
-        auto kern = merge_kernel<false>;
+template <int FMT, int NT>
+static cudaError_t launch_score_t(const ScoreArgs& a, cudaStream_t stream) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    auto kern = index_score_kernel<FMT, NT>;
+    constexpr size_t smem = score_smem_bytes<FMT>();
+    int& occ = g_score_occ[dev & 63][FMT][NT - 1];
+    if (!occ) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<dim3(ng, T), kMergeThreads, smem, stream>>>(src, (int)n, kMergeMax, k, dst, nullptr, nullptr);
-        *launches += 1;
-        n = (int64_t)ng * k;
-        uint64_t* tmp = src;
-        src = dst;
-        dst = tmp;
+        int o = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kScoreCta, smem) != cudaSuccess || o <= 0) o = 1;
+        occ = o;
     }
-    int P = 1;
-    while (P < k) P <<= 1;
-    const size_t smem = (size_t)n * 8 + 256 * 4 + 32 + (size_t)P * 8;
-    auto kern = merge_kernel<true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<dim3(1, T), kMergeThreads, smem, stream>>>(src, (int)n, (int)n, k, nullptr, out_idx, out_score);
-    *launches += 1;
+    const int64_t U = (int64_t)a.T * a.units_per_q;
+    const int64_t grid = std::min<int64_t>(U, (int64_t)sm_count(dev) * occ);
+    if (grid <= 0) return cudaSuccess;
+    kern<<<(unsigned)grid, kScoreCta, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
+                               const void* kidx, int fmt, const float* kscale, int64_t kstride_elems, int64_t sstride,
+                               int m, int max_blocks, int k, float* scores, int64_t ld_scores, unsigned* hist,
+                               unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream, int* launches) {
+    ScoreArgs a;
+    a.q = q;
+    a.w = w;
+    a.q_seq = q_seq;
+    a.q_pos = q_pos;
+    a.T = T;
+    a.Hi = Hi;
+    a.m = m;
+    a.max_blocks = max_blocks;
+    a.kidx = reinterpret_cast<const uint8_t*>(kidx);
+    a.kscale = kscale;
+    a.kstride_bytes = kstride_elems * (fmt == 0 ? 2 : 1);
+    a.sstride = sstride;
+    a.scores = scores;
+    a.ld_scores = ld_scores;
+    a.hist = hist;
+    a.done = done;
+    a.thr = thr;
+    a.status = status;
+    a.k = k;
+    a.units_per_q = (max_blocks + kUnit - 1) / kUnit;
+    const int nt = Hi > 8 ? 2 : 1;
+    cudaError_t e;
+    if (fmt == 0) e = nt == 1 ? launch_score_t<0, 1>(a, stream) : launch_score_t<0, 2>(a, stream);
+    else e = nt == 1 ? launch_score_t<1, 1>(a, stream) : launch_score_t<1, 2>(a, stream);
+    *launches += 1;
+    return e;
+}
+
+cudaError_t launch_index_select_tail(const float* scores, int64_t ld_scores, const unsigned* thr, const int* q_pos,
+                                     int T, int m, int max_blocks, int k, uint64_t* cand, int64_t cand_cap,
+                                     unsigned* cnt, int* out_idx, float* out_score, cudaStream_t stream,
+                                     int* launches) {
+    dim3 g1((max_blocks + kCollectKeys - 1) / kCollectKeys, T);
+    collect_kernel<<<g1, 256, 0, stream>>>(scores, ld_scores, thr, q_pos, m, max_blocks, cand, cand_cap, cnt);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t rank_smem = (size_t)(kRankCap + k) * 8;
+    e = cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem);
+    if (e != cudaSuccess) return e;
+    rank_kernel<<<dim3(kRankCtas, T), kRankThreads, rank_smem, stream>>>(cand, cand_cap, cnt, k, out_idx, out_score);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    *launches += 2;
+    return e;
 }
 
 }  // namespace csa

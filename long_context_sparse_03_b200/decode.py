@@ -20,7 +20,8 @@ class CsaDecoder:
     def __init__(self, inp: Inputs, kidx_fmt: int = csa.FMT_BF16, stream: torch.cuda.Stream | None = None):
         w = inp.w
         self.inp, self.w, self.fmt = inp, w, kidx_fmt
-        self.stream = stream or torch.cuda.current_stream()
+        # None = the caller's current stream at each call (graph capture works)
+        self.stream = stream
         dev = inp.raw_kv.device
         self.T = inp.T
         self.N = w.max_blocks
@@ -65,7 +66,8 @@ class CsaDecoder:
                                   kidx_scale=self.kscale, stream=self.stream)
 
     def merge(self):
-        csa.csa_index_stage_merge(self.T, self.N, self.w.k, self.idx, self.idx_score, self.ws_sel, stream=self.stream)
+        csa.csa_index_stage_merge(self.inp.q_pos, self.w.m, self.N, self.w.k, self.idx, self.idx_score, self.ws_sel,
+                                  stream=self.stream)
 
     def attend(self):
         i, w = self.inp, self.w
@@ -77,16 +79,19 @@ class CsaDecoder:
         # the stage calls lay their candidates out from the workspace header
         return self.ws_idx
 
+    def _s(self):
+        return self.stream or torch.cuda.current_stream()
+
     def step(self, ev_score: tuple | None = None):
         """One decode step on device-resident inputs.  ev_score: optional
         (start, end) CUDA events recorded around the scoring kernel."""
         self.refresh()
         self.query()
         if ev_score:
-            ev_score[0].record(self.stream)
+            ev_score[0].record(self._s())
         self.score()
         if ev_score:
-            ev_score[1].record(self.stream)
+            ev_score[1].record(self._s())
         self.merge()
         self.attend()
         return self.out
@@ -95,16 +100,23 @@ class CsaDecoder:
         """The same step from pinned host buffers: copy this step's inputs
         (hidden states, attention queries, the new token's raw rows) to the
         device, run the step, copy the attention output back."""
-        i, s = self.inp, self.stream
-        with torch.cuda.stream(s):
+        i = self.inp
+        if not hasattr(self, "_rows"):
+            dev = i.raw_kv.device
+            self._pos = (i.lens.long() - 1).to(dev)
+            self._bidx = torch.arange(self.w.B, device=dev)
+            self._kv_rows = torch.empty(kv_row_host.shape, dtype=kv_row_host.dtype, device=dev)
+            self._ki_rows = torch.empty(ki_row_host.shape, dtype=ki_row_host.dtype, device=dev)
+            self._rows = True
+        with torch.cuda.stream(self._s()):
             i.h.copy_(h_host, non_blocking=True)
             i.q.copy_(q_host, non_blocking=True)
-            pos = i.lens.long() - 1
-            bidx = torch.arange(self.w.B, device=i.raw_kv.device)
-            i.raw_kv[bidx, pos] = kv_row_host.to(i.raw_kv.device, non_blocking=True)
-            i.raw_ki[bidx, pos] = ki_row_host.to(i.raw_ki.device, non_blocking=True)
+            self._kv_rows.copy_(kv_row_host, non_blocking=True)
+            self._ki_rows.copy_(ki_row_host, non_blocking=True)
+            i.raw_kv.index_put_((self._bidx, self._pos), self._kv_rows)
+            i.raw_ki.index_put_((self._bidx, self._pos), self._ki_rows)
         self.step()
-        with torch.cuda.stream(s):
+        with torch.cuda.stream(self._s()):
             out_host.copy_(self.out, non_blocking=True)
         return out_host
 
@@ -126,7 +138,7 @@ class HcaDecoder:
     def __init__(self, inp: Inputs, stream: torch.cuda.Stream | None = None):
         w = inp.w
         self.inp, self.w = inp, w
-        self.stream = stream or torch.cuda.current_stream()
+        self.stream = stream
         dev = inp.raw_kv.device
         self.T = inp.T
         self.N = w.max_blocks
@@ -134,7 +146,7 @@ class HcaDecoder:
         self.comp = torch.empty((w.B, self.N, 128), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty((self.T, w.H, 128), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((self.T, w.H), dtype=torch.float32, device=dev)
-        self.ws_att = csa.Workspace(csa.csa_attend_workspace_size(self.T, w.H, self.N + w.W), dev, self.stream)
+        self.ws_att = csa.Workspace(csa.hca_attend_workspace_size(self.T, w.H, self.N + w.W), dev, self.stream)
 
     def build_caches(self):
         i, w = self.inp, self.w
@@ -142,13 +154,14 @@ class HcaDecoder:
 
     def step(self, ev_attend: tuple | None = None):
         i, w = self.inp, self.w
+        s = self.stream or torch.cuda.current_stream()
         csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, -1, 1, self.comp, stream=self.stream)
         if ev_attend:
-            ev_attend[0].record(self.stream)
+            ev_attend[0].record(s)
         csa.hca_attend(i.q, i.q_seq, i.q_pos, self.comp, i.raw_kv, w.m, self.N, w.W, self.scale, self.out, self.lse,
                        self.ws_att, stream=self.stream)
         if ev_attend:
-            ev_attend[1].record(self.stream)
+            ev_attend[1].record(s)
         return self.out
 
     def algorithmic_bytes(self) -> dict:

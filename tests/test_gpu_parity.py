@@ -280,7 +280,7 @@ def test_hca_attend(oracle, H, W, T, mp):
     ref, rlse = oracle.hca_attend(q, q_seq, q_pos, comp, raw, mp, W, scale)
     out = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((T, H), dtype=torch.float32, device="cuda")
-    ws = csa.Workspace(csa.csa_attend_workspace_size(T, H, N + W))
+    ws = csa.Workspace(csa.hca_attend_workspace_size(T, H, N + W))
     csa.hca_attend(dev_bf16(q), dev_i32(q_seq), dev_i32(q_pos), dev_bf16(comp), dev_bf16(raw), mp, N, W, scale, out,
                    lse, ws)
     check_attention(bf16_bits_to_f64(host_bits(out)), lse.cpu().numpy().astype(np.float64), ref, rlse)
@@ -349,3 +349,29 @@ def test_batch_invariance_and_determinism(oracle):
         alone = run(np.array([t]))
         for a, b in zip(full, alone):
             assert np.array_equal(a[t], b[0], equal_nan=True)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_index_select_all_ties(oracle, fmt):
+    """Every score equal (w = 0): the top-k is the k smallest visible block
+    indices, in order -- the candidate list then holds every block (> 8192),
+    which exercises the long-list selection path."""
+    rng = np.random.default_rng(91)
+    m, N, Hi, T, k = 4, 12000, 8, 3, 700
+    keys, ks, q, _, q_seq, q_pos = _index_case(oracle, rng, 2, N, Hi, T, fmt)
+    w = np.zeros((T, Hi), np.float32)
+    q_pos[:] = [N * m - 1, 2000, 36000]
+    kd = torch.from_numpy(keys).cuda() if fmt == 1 else dev_bf16(keys)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_index_workspace_size(T, 0, Hi, k, N))
+    csa.csa_index_select(torch.from_numpy(q).cuda(), torch.from_numpy(w).cuda(), dev_i32(q_seq), dev_i32(q_pos), kd, m,
+                         N, k, idx, sc, ws, kidx_scale=None if ks is None else torch.from_numpy(ks).cuda())
+    ws.check()
+    gi = idx.cpu().numpy()
+    for t in range(T):
+        V = min((q_pos[t] + 1) // m, N)
+        n = min(k, V)
+        assert np.array_equal(gi[t, :n], np.arange(n)), t
+        assert (gi[t, n:] == -1).all()
+        assert (sc[t, :n].cpu().numpy() == 0).all()
