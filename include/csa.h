@@ -265,6 +265,44 @@ CSA_API csa_status hca_attend(const void* q, const int32_t* q_seq, const int32_t
                       int W, float scale, void* out, float* lse,
                       void* ws, size_t ws_bytes, csa_stream_t stream);
 
+/* ------------------------------------------------------------------ */
+/* 4. Attention for callers that cannot allocate device memory.          */
+/* ------------------------------------------------------------------ */
+/*
+ * The pages have no counterpart to this call: it is a property of this
+ * library's interface, not of the method.
+ *
+ * csa_sparse_attend_noalloc computes exactly what csa_sparse_attend computes
+ * (same arguments, same kernels, same results) but takes no workspace: its
+ * split-K scratch is a fixed 16 MiB array of device memory inside the library
+ * (a static __device__ array, present on every GPU that loads the library
+ * until the process exits).  It is meant for callers that may not allocate
+ * device memory at all -- e.g. a plug-in running inside a host framework
+ * that owns every device allocation through its own pool and forbids direct
+ * cudaMalloc, or a serving loop that must never enter the driver's allocator
+ * (cudaMalloc / cudaFree can synchronise the device).  The call itself
+ * allocates nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Calls whose scratch need exceeds CSA_NOALLOC_SCRATCH_BYTES return
+ *     CSA_ERR_WORKSPACE with the sizes in csa_last_error().  The need is
+ *     the csa_attend_workspace_size(T, H, k + W) figure (about
+ *     T * ceil((k + W) / 64) * H * 520 bytes).
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents: calls that may overlap on the GPU (different streams,
+ *     or host threads) race and give wrong results; serialise them.
+ *   - Out-of-range block indices are skipped, as in csa_sparse_attend, but
+ *     no status word is set (there is no workspace to hold one).
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+CSA_API csa_status csa_sparse_attend_noalloc(const void* q, const int32_t* q_seq,
+                                             const int32_t* q_pos, int T, int H,
+                                             const void* comp, int64_t comp_seq_stride,
+                                             const void* raw, int64_t raw_seq_stride, int m,
+                                             const int32_t* idx, int k, int W, float scale,
+                                             void* out, float* lse, csa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

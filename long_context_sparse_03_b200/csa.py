@@ -22,6 +22,7 @@ HEADER = _HERE.parent / "include" / "csa.h"
 FMT_BF16 = 0
 FMT_FP8E4M3 = 1
 WS_HEADER_BYTES = 256
+NOALLOC_SCRATCH_BYTES = 16 << 20   # CSA_NOALLOC_SCRATCH_BYTES in include/csa.h
 
 STATUS = {0: "CSA_OK", 1: "CSA_ERR_NULL", 2: "CSA_ERR_SHAPE", 3: "CSA_ERR_UNSUPPORTED",
           4: "CSA_ERR_WORKSPACE", 5: "CSA_ERR_CUDA", 6: "CSA_ERR_TIMEOUT", 7: "CSA_ERR_DEVICE",
@@ -54,6 +55,7 @@ _SIGS = {
     "hca_attend_workspace_size": (_S, [_I, _I, _I]),
     "csa_sparse_attend": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _P, _I, _I, _F, _P, _P, _P, _S, _P]),
     "hca_attend": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _I, _I, _F, _P, _P, _P, _S, _P]),
+    "csa_sparse_attend_noalloc": (_I, [_P, _P, _P, _I, _I, _P, _L, _P, _L, _I, _P, _I, _I, _F, _P, _P, _P]),
 }
 
 _lib = None
@@ -232,6 +234,19 @@ def hca_attend(q, q_seq, q_pos, comp, raw, m, max_blocks, W, scale, out, lse, ws
                           raw.stride(0), m, max_blocks, W, float(scale), _ptr(out), _ptr(lse), ws.ptr(), ws.nbytes,
                           _stream(stream))
     _check(st, "hca_attend")
+    return out, lse
+
+
+def csa_sparse_attend_noalloc(q, q_seq, q_pos, comp, raw, m, idx, W, scale, out, lse, stream=None):
+    """csa_sparse_attend without a workspace: the library's fixed device
+    scratch is used instead (for callers that may not allocate device
+    memory; calls that overlap on the GPU race on that scratch)."""
+    T, H, _ = q.shape
+    k = idx.shape[1]
+    st = lib().csa_sparse_attend_noalloc(_ptr(q), _ptr(q_seq), _ptr(q_pos), T, H, _ptr(comp), comp.stride(0),
+                                         _ptr(raw), raw.stride(0), m, _ptr(idx), k, W, float(scale), _ptr(out),
+                                         _ptr(lse), _stream(stream))
+    _check(st, "csa_sparse_attend_noalloc")
     return out, lse
 
 

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/csa.h"
 #include "common.cuh"
@@ -412,6 +413,75 @@ csa_status hca_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
     REQUIRE(max_blocks >= 0, CSA_ERR_SHAPE, "max_blocks = %d < 0", max_blocks);
     return attend_common("hca_attend", q, q_seq, q_pos, T, H, comp, comp_seq_stride, raw, raw_seq_stride, m, nullptr,
                          0, max_blocks, W, scale, out, lse, ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- attention without allocation
+// csa_sparse_attend_noalloc: the same attention as csa_sparse_attend, with its
+// split-K scratch in a fixed array of device memory that belongs to the
+// library instead of a caller-supplied workspace.  For callers that may not
+// allocate device memory at all (see include/csa.h).
+constexpr size_t kNoAllocScratchBytes = CSA_NOALLOC_SCRATCH_BYTES;   // 16 MiB on every GPU that loads the library
+static __device__ __align__(256) unsigned char g_attend_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[256];   // device address of g_attend_scratch, per device ordinal
+
+// The host-side name g_attend_scratch is only a stand-in for the array; its
+// device address is looked up once per device, with that device current.
+csa_status scratch_address(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "csa_sparse_attend_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= 256) return fail(CSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attend_scratch);
+        if (e != cudaSuccess || !p) return cuda_fail(e, "csa_sparse_attend_noalloc: cudaGetSymbolAddress");
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return CSA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+csa_status csa_sparse_attend_noalloc(const void* q, const int32_t* q_seq, const int32_t* q_pos, int T, int H,
+                                     const void* comp, int64_t comp_seq_stride, const void* raw,
+                                     int64_t raw_seq_stride, int m, const int32_t* idx, int k, int W, float scale,
+                                     void* out, float* lse, csa_stream_t stream) {
+    REQUIRE(k >= 1 && k <= CSA_MAX_K, CSA_ERR_UNSUPPORTED, "k = %d outside 1..%d", k, CSA_MAX_K);
+    REQUIRE(T >= 0, CSA_ERR_SHAPE, "T = %d < 0", T);
+    REQUIRE(H >= 16 && H <= 128 && H % 16 == 0, CSA_ERR_UNSUPPORTED, "H = %d (16..128, multiple of 16)", H);
+    REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
+    REQUIRE(W >= 0 && W <= CSA_MAX_W, CSA_ERR_UNSUPPORTED, "W = %d outside 0..%d", W, CSA_MAX_W);
+    REQUIRE(std::isfinite(scale), CSA_ERR_SHAPE, "scale is not finite");
+    REQUIRE(comp_seq_stride >= 0 && raw_seq_stride >= 0, CSA_ERR_SHAPE, "negative stride");
+    if (T == 0) return ok();
+    REQUIRE(q && q_seq && q_pos && comp && raw && out && idx, CSA_ERR_NULL,
+            "q, q_seq, q_pos, comp, raw, idx and out are required");
+    REQUIRE(aligned16(q) && aligned16(comp) && aligned16(raw), CSA_ERR_ALIGN, "q, comp and raw must be 16-byte aligned");
+    REQUIRE(comp_seq_stride % 8 == 0 && raw_seq_stride % 8 == 0, CSA_ERR_ALIGN, "strides must be multiples of 8");
+    const AttendLayout L = attend_layout(T, H, k + W, false);
+    REQUIRE(L.total <= kNoAllocScratchBytes, CSA_ERR_WORKSPACE,
+            "this call needs %zu bytes of scratch; the fixed scratch holds %zu (use csa_sparse_attend with a "
+            "workspace for larger T, H, k + W)",
+            L.total, kNoAllocScratchBytes);
+    void* base = nullptr;
+    csa_status s = scratch_address(&base);
+    if (s != CSA_OK) return s;
+    int n = 0;
+    cudaError_t e = csa::launch_attend(q, q_seq, q_pos, T, H, comp, comp_seq_stride, raw, raw_seq_stride, m, idx, k,
+                                       0, W, scale, out, lse, reinterpret_cast<float*>((char*)base + L.part_o),
+                                       reinterpret_cast<float*>((char*)base + L.part_ml), nullptr,
+                                       (cudaStream_t)stream, &n);
+    count(n);
+    if (e != cudaSuccess) return cuda_fail(e, "csa_sparse_attend_noalloc");
+    return ok();
 }
 
 }  // extern "C"
