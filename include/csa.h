@@ -114,7 +114,7 @@ CSA_API uint64_t csa_launch_count(void);
 /* Bytes reserved at the start of every workspace for the status word. */
 #define CSA_WS_HEADER_BYTES 256
 
-/* Zero the status word of a freshly allocated workspace (async). */
+/* Zero a freshly allocated workspace (async), in particular its status word. */
 CSA_API csa_status csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream);
 
 /* Synchronise `stream`, read the workspace's status word, clear it.

@@ -24,7 +24,8 @@ cudaError_t launch_index_query(const void* h, int T, int D, int r, int Hi, const
 cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
                                const void* kidx, int fmt, const float* kscale, int64_t kstride_elems, int64_t sstride,
                                int m, int max_blocks, int k, float* scores, int64_t ld_scores, unsigned* hist,
-                               unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream, int* launches);
+                               unsigned* cnt, unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream,
+                               int* launches);
 cudaError_t launch_index_select_tail(const float* scores, int64_t ld_scores, const unsigned* thr, const int* q_pos,
                                      int T, int m, int max_blocks, int k, uint64_t* cand, int64_t cand_cap,
                                      unsigned* cnt, int* out_idx, float* out_score, cudaStream_t stream,
@@ -34,7 +35,8 @@ int attend_nsplit(int max_rows, bool dense);
 cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int T, int H, const void* comp,
                           int64_t comp_stride, const void* raw, int64_t raw_stride, int m, const int* idx, int k,
                           int max_blocks, int W, float scale, void* out, float* lse, float* part_o,
-                          float* part_ml, unsigned* status, cudaStream_t stream, int* launches);
+                          float* part_ml, unsigned* status, bool use_partials, cudaStream_t stream,
+                          int* launches);
 }  // namespace csa
 
 namespace {
@@ -71,19 +73,16 @@ size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 int64_t cand_cap(int max_blocks) { return ((int64_t)max_blocks + 1) & ~(int64_t)1; }
 
 struct IndexLayout {
-    size_t u, q, w, hist, cnt, done, thr, scores, cand, total;
+    size_t hist, cnt, done, thr, scores, cand, q, w, u, total;
 };
-// header | u [T][r] | q [T][Hi][64] | w [T][Hi] | hist [T][4096] | cnt [T] |
-// done [T] | thr [T] | scores [T][max_blocks] fp32 | cand [T][max_blocks] u64
+// header | hist [T][2048] | cnt [T] | done [T] | thr [T] | scores [T][max_blocks] fp32 |
+// cand [T][cand_cap] u64 | q [T][Hi][64] | w [T][Hi] | u [T][r].
+// The scoring pass zeroes the selection state (hist, cnt, done: contiguous)
+// itself.  csa_index_query keeps u at the very end of whatever workspace it
+// is given.
 IndexLayout index_layout(int T, int r, int Hi, int max_blocks) {
     IndexLayout L;
     size_t off = CSA_WS_HEADER_BYTES;
-    L.u = off;
-    off = up256(off + (size_t)T * r * 4);
-    L.q = off;
-    off = up256(off + (size_t)T * Hi * 64 * 4);
-    L.w = off;
-    off = up256(off + (size_t)T * Hi * 4);
     L.hist = off;
     L.cnt = off + (size_t)T * csa::kHistBins * 4;
     L.done = L.cnt + (size_t)T * 4;
@@ -93,6 +92,12 @@ IndexLayout index_layout(int T, int r, int Hi, int max_blocks) {
     off = up256(off + (size_t)T * max_blocks * 4);
     L.cand = off;
     off = up256(off + (size_t)T * cand_cap(max_blocks) * 8);
+    L.q = off;
+    off = up256(off + (size_t)T * Hi * 64 * 4);
+    L.w = off;
+    off = up256(off + (size_t)T * Hi * 4);
+    L.u = off;
+    off = up256(off + (size_t)T * r * 4);
     L.total = off;
     return L;
 }
@@ -156,7 +161,7 @@ uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relax
 csa_status csa_workspace_init(void* ws, size_t ws_bytes, csa_stream_t stream) {
     REQUIRE(ws, CSA_ERR_NULL, "ws is NULL");
     REQUIRE(ws_bytes >= CSA_WS_HEADER_BYTES, CSA_ERR_WORKSPACE, "workspace smaller than its header");
-    cudaError_t e = cudaMemsetAsync(ws, 0, CSA_WS_HEADER_BYTES, (cudaStream_t)stream);
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "csa_workspace_init");
     return ok();
 }
@@ -220,12 +225,15 @@ csa_status csa_index_query(const void* h, int T, int D, int r, int Hi, const voi
     REQUIRE(h && W_dq && W_uq && W_w && q_out && w_out && ws, CSA_ERR_NULL, "a required pointer is NULL");
     REQUIRE(aligned16(h) && aligned16(W_dq) && aligned16(W_uq) && aligned16(W_w) && aligned16(ws), CSA_ERR_ALIGN,
             "h, weights and ws must be 16-byte aligned");
-    const size_t need = CSA_WS_HEADER_BYTES + up256((size_t)T * r * 4);
+    const size_t ubytes = up256((size_t)T * r * 4);
+    const size_t need = CSA_WS_HEADER_BYTES + ubytes;
     REQUIRE(ws_bytes >= need, CSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+    // u lives at the end of the workspace (256-byte aligned), clear of the
+    // selection state at its start
+    const size_t uoff = (ws_bytes - ubytes) & ~(size_t)255;
     int n = 0;
     cudaError_t e = csa::launch_index_query(h, T, D, r, Hi, W_dq, W_uq, W_w, q_out, w_out,
-                                            reinterpret_cast<float*>((char*)ws + CSA_WS_HEADER_BYTES),
-                                            (cudaStream_t)stream, &n);
+                                            reinterpret_cast<float*>((char*)ws + uoff), (cudaStream_t)stream, &n);
     count(n);
     if (e != cudaSuccess) return cuda_fail(e, "csa_index_query");
     return ok();
@@ -245,7 +253,7 @@ csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq
     if (e == cudaSuccess)
         e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
                                     scale_seq_stride, m, max_blocks, 1, scores, max_blocks, nullptr, nullptr,
-                                    nullptr, nullptr, (cudaStream_t)stream, &n);
+                                    nullptr, nullptr, nullptr, (cudaStream_t)stream, &n);
     count(n);
     if (e != cudaSuccess) return cuda_fail(e, "csa_index_scores");
     return ok();
@@ -256,15 +264,15 @@ static csa_status stage_score(const char* who, const float* q, const float* w, c
                               const float* kidx_scale, int64_t kidx_seq_stride, int64_t scale_seq_stride, int m,
                               int max_blocks, int k, const IndexLayout& L, void* ws, cudaStream_t stream) {
     char* base = (char*)ws;
-    cudaError_t e = cudaMemsetAsync(base + L.hist, 0, L.scores - L.hist, stream);  // hist, cnt, done, thr
     int n = 0;
-    if (e == cudaSuccess)
-        e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
-                                    scale_seq_stride, m, max_blocks, k, reinterpret_cast<float*>(base + L.scores),
-                                    max_blocks, reinterpret_cast<unsigned*>(base + L.hist),
-                                    reinterpret_cast<unsigned*>(base + L.done),
-                                    reinterpret_cast<unsigned*>(base + L.thr), reinterpret_cast<unsigned*>(base),
-                                    stream, &n);
+    cudaError_t e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
+                                            scale_seq_stride, m, max_blocks, k,
+                                            reinterpret_cast<float*>(base + L.scores), max_blocks,
+                                            reinterpret_cast<unsigned*>(base + L.hist),
+                                            reinterpret_cast<unsigned*>(base + L.cnt),
+                                            reinterpret_cast<unsigned*>(base + L.done),
+                                            reinterpret_cast<unsigned*>(base + L.thr), reinterpret_cast<unsigned*>(base),
+                                            stream, &n);
     count(n);
     if (e != cudaSuccess) return cuda_fail(e, who);
     return ok();
@@ -391,7 +399,7 @@ static csa_status attend_common(const char* who, const void* q, const int32_t* q
                                        max_blocks, W, scale, out, lse,
                                        reinterpret_cast<float*>((char*)ws + L.part_o),
                                        reinterpret_cast<float*>((char*)ws + L.part_ml),
-                                       reinterpret_cast<unsigned*>(ws), (cudaStream_t)stream, &n);
+                                       reinterpret_cast<unsigned*>(ws), false, (cudaStream_t)stream, &n);
     count(n);
     if (e != cudaSuccess) return cuda_fail(e, who);
     return ok();
@@ -477,7 +485,7 @@ csa_status csa_sparse_attend_noalloc(const void* q, const int32_t* q_seq, const 
     int n = 0;
     cudaError_t e = csa::launch_attend(q, q_seq, q_pos, T, H, comp, comp_seq_stride, raw, raw_seq_stride, m, idx, k,
                                        0, W, scale, out, lse, reinterpret_cast<float*>((char*)base + L.part_o),
-                                       reinterpret_cast<float*>((char*)base + L.part_ml), nullptr,
+                                       reinterpret_cast<float*>((char*)base + L.part_ml), nullptr, true,
                                        (cudaStream_t)stream, &n);
     count(n);
     if (e != cudaSuccess) return cuda_fail(e, "csa_sparse_attend_noalloc");

@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
 
     const int t = blockIdx.y, sp = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    griddep_wait();
     const int b = a.q_seq[t], p = a.q_pos[t];
     const int V = a.idx ? (p + 1) / a.m : min((p + 1) / a.m, a.max_blocks);
     const int nsel = a.idx ? a.k : V;
@@ -229,70 +230,67 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
         pm[(h0 + 8) * 2] = mrow[1];
         pm[(h0 + 8) * 2 + 1] = lrow[1];
     }
+    griddep_trigger();
 }
 
-// grid (H, T), 128 threads (one per output channel).  The splits' (max, sum)
-// pairs are staged once in shared memory; each thread then issues all its
-// partial-output loads before combining them in split order.
-constexpr int kCombineMaxSplits = 512;
+// Merge of the split partials of one (query, head) per warp: lane i holds
+// split i's (max, sum) -- 32 splits per pass, passes merged in order -- and
+// every lane owns 4 output channels, issuing all its splits' partial-output
+// loads before summing them in split order.  grid (H / 4, T), 128 threads.
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                                       int nsplit, int H, bf16* __restrict__ out,
                                                       float* __restrict__ lse) {
-    __shared__ float fac[kCombineMaxSplits];
-    __shared__ float red[2];
-    const int h = blockIdx.x, t = blockIdx.y, c = threadIdx.x;
-    // global max over the splits (fixed order reduction: per-thread then warp tree)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x * 4 + warp, t = blockIdx.y;
+    griddep_wait();
+    if (h >= H) return;
+    // pass 1: the global max
     float M = -INFINITY;
-    for (int i = c; i < nsplit; i += 128) {
-        const float mi = part_ml[(((int64_t)t * nsplit + i) * H + h) * 2];
-        if (i < kCombineMaxSplits) fac[i] = mi;
+    for (int base = 0; base < nsplit; base += 32) {
+        const int i = base + lane;
+        const float mi = i < nsplit ? part_ml[(((int64_t)t * nsplit + i) * H + h) * 2] : -INFINITY;
         M = fmaxf(M, mi);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    __shared__ float wm[4];
-    if ((c & 31) == 0) wm[c >> 5] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
-    // per-split factors 2^(m_i - M) (0 for empty splits)
-    for (int i = c; i < nsplit && i < kCombineMaxSplits; i += 128) {
-        const float mi = fac[i];
-        fac[i] = (M == -INFINITY || mi == -INFINITY) ? 0.f : exp2f(mi - M);
-    }
-    __syncthreads();
-    if (c == 0) {
-        float L = 0.f;
-        for (int i = 0; i < nsplit; ++i) {
-            const float f = i < kCombineMaxSplits ? fac[i]
-                                                  : ((M == -INFINITY) ? 0.f
-                                                                      : exp2f(part_ml[(((int64_t)t * nsplit + i) * H + h) * 2] - M));
-            L = fmaf(part_ml[(((int64_t)t * nsplit + i) * H + h) * 2 + 1], f, L);
+    // pass 2: factors, sum and output, 32 splits at a time in split order
+    float L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int base = 0; base < nsplit; base += 32) {
+        const int i = base + lane;
+        float f = 0.f, li = 0.f;
+        if (i < nsplit) {
+            const int64_t o = (((int64_t)t * nsplit + i) * H + h) * 2;
+            const float mi = part_ml[o];
+            li = part_ml[o + 1];
+            f = (M == -INFINITY || mi == -INFINITY) ? 0.f : exp2f(mi - M);
         }
-        red[0] = L;
+        const int cnt = min(32, nsplit - base);
+        float4 ov[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < cnt)
+                ov[j] = *reinterpret_cast<const float4*>(part_o + (((int64_t)t * nsplit + base + j) * H + h) * 128 +
+                                                         lane * 4);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if (j < cnt) {
+                const float fj = __shfl_sync(0xffffffffu, f, j);
+                const float lj = __shfl_sync(0xffffffffu, li, j);
+                L = fmaf(lj, fj, L);
+                O.x = fmaf(ov[j].x, fj, O.x);
+                O.y = fmaf(ov[j].y, fj, O.y);
+                O.z = fmaf(ov[j].z, fj, O.z);
+                O.w = fmaf(ov[j].w, fj, O.w);
+            }
+        }
     }
-    float O = 0.f;
-    int i = 0;
-    for (; i + 4 <= nsplit && i + 4 <= kCombineMaxSplits; i += 4) {   // four loads in flight
-        const float o0 = part_o[(((int64_t)t * nsplit + i) * H + h) * 128 + c];
-        const float o1 = part_o[(((int64_t)t * nsplit + i + 1) * H + h) * 128 + c];
-        const float o2 = part_o[(((int64_t)t * nsplit + i + 2) * H + h) * 128 + c];
-        const float o3 = part_o[(((int64_t)t * nsplit + i + 3) * H + h) * 128 + c];
-        O = fmaf(o0, fac[i], O);
-        O = fmaf(o1, fac[i + 1], O);
-        O = fmaf(o2, fac[i + 2], O);
-        O = fmaf(o3, fac[i + 3], O);
-    }
-    for (; i < nsplit; ++i) {
-        const float f = i < kCombineMaxSplits ? fac[i]
-                                              : ((M == -INFINITY) ? 0.f
-                                                                  : exp2f(part_ml[(((int64_t)t * nsplit + i) * H + h) * 2] - M));
-        O = fmaf(part_o[(((int64_t)t * nsplit + i) * H + h) * 128 + c], f, O);
-    }
-    __syncthreads();
-    const float L = red[0];
-    const float res = L > 0.f ? O / L : 0.f;
-    out[((int64_t)t * H + h) * 128 + c] = __float2bfloat16_rn(res);
-    if (lse && c == 0) lse[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    bf16* op = out + ((int64_t)t * H + h) * 128 + lane * 4;
+    const float r0 = L > 0.f ? O.x / L : 0.f, r1 = L > 0.f ? O.y / L : 0.f;
+    const float r2 = L > 0.f ? O.z / L : 0.f, r3 = L > 0.f ? O.w / L : 0.f;
+    *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16(r0, r1), pack_bf16(r2, r3));
+    if (lse && lane == 0) lse[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    griddep_trigger();
 }
 
 int attend_rows_per_split(bool dense) { return dense ? kHcaRowsPerSplit : kCsaRowsPerSplit; }
@@ -304,7 +302,9 @@ int attend_nsplit(int max_rows, bool dense) {
 cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int T, int H, const void* comp,
                           int64_t comp_stride, const void* raw, int64_t raw_stride, int m, const int* idx, int k,
                           int max_blocks, int W, float scale, void* out, float* lse, float* part_o,
-                          float* part_ml, unsigned* status, cudaStream_t stream, int* launches) {
+                          float* part_ml, unsigned* status, bool use_partials, cudaStream_t stream,
+                          int* launches) {
+    (void)use_partials;   // every split writes partials that combine_kernel merges
     AttnArgs a;
     a.q = reinterpret_cast<const bf16*>(q);
     a.q_seq = q_seq;
@@ -326,20 +326,23 @@ cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int
     a.part_ml = part_ml;
     a.status = status;
     dim3 grid(a.nsplit, T);
+    cudaError_t e = cudaSuccess;
     switch (H) {
-        case 16: attend_kernel<1><<<grid, 32, 0, stream>>>(a); break;
-        case 32: attend_kernel<2><<<grid, 64, 0, stream>>>(a); break;
-        case 48: attend_kernel<3><<<grid, 96, 0, stream>>>(a); break;
-        case 64: attend_kernel<4><<<grid, 128, 0, stream>>>(a); break;
-        case 80: attend_kernel<5><<<grid, 160, 0, stream>>>(a); break;
-        case 96: attend_kernel<6><<<grid, 192, 0, stream>>>(a); break;
-        case 112: attend_kernel<7><<<grid, 224, 0, stream>>>(a); break;
-        case 128: attend_kernel<8><<<grid, 256, 0, stream>>>(a); break;
+        case 16: e = launch_pdl(attend_kernel<1>, grid, dim3(32), 0, stream, a); break;
+        case 32: e = launch_pdl(attend_kernel<2>, grid, dim3(64), 0, stream, a); break;
+        case 48: e = launch_pdl(attend_kernel<3>, grid, dim3(96), 0, stream, a); break;
+        case 64: e = launch_pdl(attend_kernel<4>, grid, dim3(128), 0, stream, a); break;
+        case 80: e = launch_pdl(attend_kernel<5>, grid, dim3(160), 0, stream, a); break;
+        case 96: e = launch_pdl(attend_kernel<6>, grid, dim3(192), 0, stream, a); break;
+        case 112: e = launch_pdl(attend_kernel<7>, grid, dim3(224), 0, stream, a); break;
+        case 128: e = launch_pdl(attend_kernel<8>, grid, dim3(256), 0, stream, a); break;
         default: return cudaErrorInvalidValue;
     }
-    combine_kernel<<<dim3(H, T), 128, 0, stream>>>(part_o, part_ml, a.nsplit, H, reinterpret_cast<bf16*>(out), lse);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(combine_kernel, dim3((H + 3) / 4, T), dim3(128), 0, stream, (const float*)part_o,
+                   (const float*)part_ml, a.nsplit, H, reinterpret_cast<bf16*>(out), lse);
     *launches += 2;
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace csa

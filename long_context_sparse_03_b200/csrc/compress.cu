@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) compress_kernel(
     constexpr int RPC = 256 / TPR;        // output rows per CTA
     extern __shared__ float a_sh[];       // [m][D] pooling weights
 
+    griddep_wait();
     for (int c = threadIdx.x; c < D; c += blockDim.x) {
         float mx = -INFINITY;
         for (int i = 0; i < m; ++i) mx = fmaxf(mx, logits[i * D + c]);
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(256) compress_kernel(
         *reinterpret_cast<uint2*>(dst) = codes;
         if (chunk == 0) out_scale[(int64_t)b * scale_stride + j] = s;
     }
+    griddep_trigger();
 }
 
 // Launch: grid.x covers the requested block range, grid.y the sequences.
@@ -120,20 +122,23 @@ cudaError_t launch_compress(const void* raw, int64_t raw_stride, const int* lens
         auto k = compress_kernel<128, 0>;
         if (smem > 48 * 1024) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<grid, 256, smem, stream>>>(r, raw_stride, lens, m, logits, blk_lo, blk_hi, out, out_stride,
-                                       out_scale, scale_stride);
+        e = launch_pdl(k, grid, dim3(256), smem, stream, r, raw_stride, lens, m, logits, blk_lo, blk_hi, out,
+                       out_stride, out_scale, scale_stride);
+        if (e != cudaSuccess) return e;
     } else if (out_fmt == 0) {
         auto k = compress_kernel<64, 0>;
         if (smem > 48 * 1024) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<grid, 256, smem, stream>>>(r, raw_stride, lens, m, logits, blk_lo, blk_hi, out, out_stride,
-                                       out_scale, scale_stride);
+        e = launch_pdl(k, grid, dim3(256), smem, stream, r, raw_stride, lens, m, logits, blk_lo, blk_hi, out,
+                       out_stride, out_scale, scale_stride);
+        if (e != cudaSuccess) return e;
     } else {
         auto k = compress_kernel<64, 1>;
         if (smem > 48 * 1024) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        k<<<grid, 256, smem, stream>>>(r, raw_stride, lens, m, logits, blk_lo, blk_hi, out, out_stride,
-                                       out_scale, scale_stride);
+        e = launch_pdl(k, grid, dim3(256), smem, stream, r, raw_stride, lens, m, logits, blk_lo, blk_hi, out,
+                       out_stride, out_scale, scale_stride);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

@@ -77,6 +77,7 @@ __global__ void __launch_bounds__(kGemvRows * 32) gemv_kernel(const bf16* __rest
         ld = ld1;
     }
     const int nchunk = K / 8;
+    griddep_wait();
     for (int t0 = 0; t0 < T; t0 += kGemvTT) {
         __syncthreads();
         stage_x<XT>(xs, X, T, t0, K);
@@ -118,6 +119,119 @@ __global__ void __launch_bounds__(kGemvRows * 32) gemv_kernel(const bf16* __rest
             if (lane == 0 && t0 + u < T) yr[(int64_t)(t0 + u) * ld] = v;
         }
     }
+    griddep_trigger();
+}
+
+// ---------------------------------------------------------------- tensor-core GEMV
+// Y[t][row] = sum_c W[row][c] X[t][c] for bf16 W and bf16 X (exact bf16
+// products, fp32 accumulation) on mma.m16n8k16: a warp takes 16 weight rows
+// as the A operand, loaded straight from global memory into registers
+// (lane quarter tq holds 16-byte chunks tq and tq+4 of every 64-element
+// block of rows g and g+8), and up to 8 queries as B, read from the staged
+// copy of X with the same channel permutation.  The CTA's 16 warps split K
+// evenly; their 16 x 8 partial tiles are summed in warp order (fixed, so
+// deterministic).  Used when K is a multiple of 1024 (64 channels x 16
+// warps); other K use the SIMT kernel above.
+constexpr int kMmaWarps = 16;
+
+// Stage X[t0 .. t0+8)[0..K) (bf16) into shared memory already laid out as
+// B fragments: the 8 bytes lane (g, tq) needs for k-step s of 64-channel
+// block b -- channels b*64 + (s>>1)*32 + tq*8 + (s&1)*4 .. +4 of query g --
+// sit at 8-byte slot ((b*4 + s)*4 + tq)*8 + g, so a warp's fragment load is
+// 256 contiguous bytes (no bank conflicts).  Queries past T read as zero.
+__device__ __forceinline__ void stage_x_frag(uint2* xs, const bf16* X, int T, int t0, int K) {
+    const int nslot = (K / 4) * kGemvTT;   // 8-byte slots
+    for (int i = threadIdx.x; i < nslot; i += blockDim.x) {
+        const int g = i & 7, tq = (i >> 3) & 3, s = (i >> 5) & 3, b = i >> 7;
+        const int c = b * 64 + (s >> 1) * 32 + tq * 8 + (s & 1) * 4;
+        const bool ok = t0 + g < T;
+        const uint32_t d = (uint32_t)__cvta_generic_to_shared(xs + i);
+        const void* src = ok ? (const void*)(X + (int64_t)(t0 + g) * K + c) : (const void*)X;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n" ::"r"(d), "l"(src), "r"(ok ? 8 : 0));
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+}
+
+__global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(const bf16* __restrict__ W0, int n0,
+                                                                 float* __restrict__ Y0, int ld0,
+                                                                 const bf16* __restrict__ W1, int n1,
+                                                                 float* __restrict__ Y1, int ld1, int K,
+                                                                 const bf16* __restrict__ X, int T) {
+    extern __shared__ __align__(16) uint8_t smem_g[];
+    uint2* xs = reinterpret_cast<uint2*>(smem_g);                                 // B fragments, 16 * K bytes
+    float* part = reinterpret_cast<float*>(smem_g + (size_t)kGemvTT * K * 2);     // [kMmaWarps][16][8]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int row0 = blockIdx.x * 16;
+    const int KW = K / kMmaWarps;               // channels per warp (multiple of 64)
+    const int c_lo = warp * KW;
+    // the two weight rows of this lane (rows past n0 + n1 read as zero)
+    auto wrow = [&](int r) -> const bf16* {
+        if (r < n0) return W0 + (int64_t)r * K;
+        if (r < n0 + n1) return W1 + (int64_t)(r - n0) * K;
+        return nullptr;
+    };
+    const bf16* wa = wrow(row0 + g);
+    const bf16* wb = wrow(row0 + g + 8);
+    griddep_wait();
+    for (int t0 = 0; t0 < T; t0 += kGemvTT) {
+        __syncthreads();
+        stage_x_frag(xs, X, T, t0, K);
+        __syncthreads();
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int cb = c_lo; cb < c_lo + KW; cb += 256) {
+            // four 64-channel blocks: 16 loads of 16 bytes in flight per lane
+            uint4 a[4][4];
+            const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int bk = 0; bk < 4; ++bk) {
+                const int cc = cb + bk * 64;
+                const bool in = cc < c_lo + KW;
+                a[bk][0] = (in && wa) ? ldg_stream(wa + cc + tq * 8) : z;        // row g, chunk tq
+                a[bk][1] = (in && wa) ? ldg_stream(wa + cc + 32 + tq * 8) : z;   // row g, chunk tq+4
+                a[bk][2] = (in && wb) ? ldg_stream(wb + cc + tq * 8) : z;        // row g+8, chunk tq
+                a[bk][3] = (in && wb) ? ldg_stream(wb + cc + 32 + tq * 8) : z;   // row g+8, chunk tq+4
+            }
+#pragma unroll
+            for (int bk = 0; bk < 4; ++bk) {
+                const int cc = cb + bk * 64;
+                if (cc >= c_lo + KW) break;
+                const uint2* xb = xs + (size_t)(cc / 64) * 128 + tq * 8 + g;
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    // channels of k-step s for lane tq: (s>>1)*32 + tq*8 + (s&1)*4 + {0..3}
+                    const uint4& A = (s < 2) ? a[bk][0] : a[bk][1];
+                    const uint4& B = (s < 2) ? a[bk][2] : a[bk][3];
+                    const bool hiw = s & 1;
+                    uint32_t af[4];
+                    af[0] = hiw ? A.z : A.x;
+                    af[2] = hiw ? A.w : A.y;
+                    af[1] = hiw ? B.z : B.x;
+                    af[3] = hiw ? B.w : B.y;
+                    const uint2 bb = xb[s * 32];
+                    mma_bf16_16816(c, af, bb.x, bb.y);
+                }
+            }
+        }
+        // c: (row g, queries 2tq, 2tq+1), (row g+8, same queries)
+        float* pw = part + warp * 128;
+        pw[g * 8 + 2 * tq] = c[0];
+        pw[g * 8 + 2 * tq + 1] = c[1];
+        pw[(g + 8) * 8 + 2 * tq] = c[2];
+        pw[(g + 8) * 8 + 2 * tq + 1] = c[3];
+        __syncthreads();
+        if (threadIdx.x < 128) {
+            const int rr = threadIdx.x >> 3, u = threadIdx.x & 7;
+            float acc = 0.f;
+            for (int w2 = 0; w2 < kMmaWarps; ++w2) acc += part[w2 * 128 + rr * 8 + u];
+            const int r = row0 + rr;
+            if (t0 + u < T) {
+                if (r < n0) Y0[(int64_t)(t0 + u) * ld0 + r] = acc;
+                else if (r < n0 + n1) Y1[(int64_t)(t0 + u) * ld1 + (r - n0)] = acc;
+            }
+        }
+    }
+    griddep_trigger();
 }
 
 template <typename XT>
@@ -129,9 +243,8 @@ static cudaError_t launch_gemv(const bf16* W0, int n0, float* Y0, int ld0, const
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    kern<<<(n0 + n1 + kGemvRows - 1) / kGemvRows, kGemvRows * 32, smem, stream>>>(W0, n0, Y0, ld0, W1, n1, Y1, ld1,
-                                                                                  K, X, T);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((n0 + n1 + kGemvRows - 1) / kGemvRows), dim3(kGemvRows * 32), smem, stream, W0, n0,
+                      Y0, ld0, W1, n1, Y1, ld1, K, X, T);
 }
 
 // q_out [T][Hi*64], w_out [T][Hi], u_ws [T][r] (fp32 scratch).
@@ -139,8 +252,18 @@ cudaError_t launch_index_query(const void* h, int T, int D, int r, int Hi, const
                                const void* W_w, float* q_out, float* w_out, float* u_ws, cudaStream_t stream,
                                int* launches) {
     const bf16* hb = reinterpret_cast<const bf16*>(h);
-    cudaError_t e = launch_gemv<bf16>(reinterpret_cast<const bf16*>(W_dq), r, u_ws, r,
-                                      reinterpret_cast<const bf16*>(W_w), Hi, w_out, Hi, D, hb, T, stream);
+    cudaError_t e;
+    if (D % (64 * kMmaWarps) == 0) {
+        const size_t smem = (size_t)kGemvTT * D * 2 + (size_t)kMmaWarps * 128 * 4;
+        e = cudaFuncSetAttribute(gemv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        e = launch_pdl(gemv_mma_kernel, dim3((r + Hi + 15) / 16), dim3(kMmaWarps * 32), smem, stream,
+                       reinterpret_cast<const bf16*>(W_dq), r, u_ws, r, reinterpret_cast<const bf16*>(W_w), Hi,
+                       w_out, Hi, D, hb, T);
+    } else {
+        e = launch_gemv<bf16>(reinterpret_cast<const bf16*>(W_dq), r, u_ws, r, reinterpret_cast<const bf16*>(W_w), Hi,
+                              w_out, Hi, D, hb, T, stream);
+    }
     if (e != cudaSuccess) return e;
     e = launch_gemv<float>(reinterpret_cast<const bf16*>(W_uq), Hi * 64, q_out, Hi * 64, nullptr, 0, nullptr, 0, r,
                            u_ws, T, stream);

@@ -46,9 +46,14 @@ constexpr int kCollectKeys = 4096;    // scores scanned per collect CTA
 // Exact threshold of the kk largest among the distinct nonzero uint64 values
 // v[0..n) (zero = empty).  Returns thr with exactly min(kk, #nonzero) values
 // >= thr among the nonzero ones (thr = 1 when every value is taken).  v may
-// be shared or global memory.  Every thread of the block must call it.
+// be shared or global memory.  Radix select from the top with 11-bit digits
+// (2048-bin shared histogram hist[2048]); it stops as soon as the boundary
+// digit holds exactly the keys still needed.  Every thread of the block must
+// call it; blockDim.x must be a multiple of 32 and at most 1024.
+constexpr int kSelBins = 2048;
 __device__ uint64_t block_select(const uint64_t* v, int n, int kk, unsigned* hist, int* misc) {
-    const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31;
+    const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarp = nth >> 5;
+    __shared__ unsigned wsum[32];
     if (tid == 0) misc[2] = 0;
     __syncthreads();
     int cnt = 0;
@@ -61,56 +66,61 @@ __device__ uint64_t block_select(const uint64_t* v, int n, int kk, unsigned* his
 
     uint64_t prefix = 0, mask = 0;
     int need = kk;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += nth) hist[i] = 0;
+    const int per = kSelBins / nth;   // bins per thread (>= 2)
+    for (int shift = 53; shift > -11; shift -= 11) {
+        const int sh = shift > 0 ? shift : 0;
+        const int width = shift > 0 ? 11 : 11 + shift;   // the last digit is the 9 low bits
+        const uint64_t dmask = ((uint64_t)1 << width) - 1;
+        for (int i = tid; i < kSelBins; i += nth) hist[i] = 0;
         __syncthreads();
-        for (int base = 0; base < n; base += nth) {
-            const int i = base + tid;
-            const uint64_t x = i < n ? v[i] : 0ull;
-            const bool match = x != 0ull && (x & mask) == prefix;
-            const unsigned dig = (unsigned)(x >> shift) & 255u;
-            const unsigned peers = __match_any_sync(0xffffffffu, match ? dig : 0xFFFFFFFFu);
-            if (match && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (unsigned)__popc(peers));
+        for (int i = tid; i < n; i += nth) {
+            const uint64_t x = v[i];
+            if (x != 0ull && (x & mask) == prefix) atomicAdd(&hist[(unsigned)((x >> sh) & dmask)], 1u);
         }
         __syncthreads();
-        if (tid < 32) {
-            // lane L owns bins 255-8L .. 248-8L (highest first)
-            unsigned c[8], s = 0;
+        // thread tid owns bins counted from the top: [tid*per, tid*per + per)
+        unsigned c[16], tot = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                c[e] = hist[255 - 8 * lane - e];
-                s += c[e];
-            }
-            unsigned incl = s;
+        for (int e = 0; e < 16; ++e) {
+            c[e] = e < per ? hist[kSelBins - 1 - (tid * per + e)] : 0u;
+            tot += c[e];
+        }
+        unsigned incl = tot;
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o;
-            }
-            const unsigned excl = incl - s;
-            if (excl < (unsigned)need && (unsigned)need <= incl) {
-                unsigned run = excl;
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        unsigned before = 0;
+        for (int w2 = 0; w2 < warp; ++w2) before += wsum[w2];
+        incl += before;
+        const unsigned excl = incl - tot;
+        if (excl < (unsigned)need && (unsigned)need <= incl) {
+            unsigned run = excl;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    if (run + c[e] >= (unsigned)need) {
-                        misc[0] = 255 - 8 * lane - e;
-                        misc[1] = (int)run;
-                        break;
-                    }
-                    run += c[e];
+            for (int e = 0; e < 16; ++e) {
+                if (e < per && run + c[e] >= (unsigned)need) {
+                    misc[0] = kSelBins - 1 - (tid * per + e);
+                    misc[1] = (int)run;
+                    misc[3] = (int)c[e];
+                    break;
                 }
+                run += c[e];
             }
         }
         __syncthreads();
-        const unsigned d = (unsigned)misc[0];
+        const uint64_t d = (uint64_t)misc[0];
         const int above = misc[1];
-        const unsigned bin = hist[d];
-        prefix |= (uint64_t)d << shift;
-        mask |= 0xFFull << shift;
+        const int bin = misc[3];
+        prefix |= d << sh;
+        mask |= dmask << sh;
         need -= above;
         __syncthreads();  // misc / hist are rewritten by the next pass
-        if ((int)bin == need) break;
+        if (bin == need) break;
     }
+    (void)nwarp;
     return prefix;
 }
 
@@ -466,6 +476,15 @@ __device__ void leave_query(const ScoreArgs& a, int t, int contributors, ScoreSm
     }
 }
 
+// Zero the per-query selection state (histograms, candidate counts, done
+// counters) that the scoring pass accumulates into.  grid-stride, 256 threads.
+__global__ void __launch_bounds__(256) zero_state_kernel(unsigned* __restrict__ state, int64_t words) {
+    griddep_wait();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words; i += (int64_t)gridDim.x * blockDim.x)
+        state[i] = 0u;
+    griddep_trigger();
+}
+
 // CTA that owns work unit x under the even split of U units over G CTAs.
 __device__ __forceinline__ int owner_cta(int64_t x, int64_t U, int64_t G) { return (int)(((x + 1) * G - 1) / U); }
 
@@ -505,6 +524,7 @@ __global__ void __launch_bounds__(kScoreCta, 2) index_score_kernel(ScoreArgs a) 
     }
     for (int i = threadIdx.x; i < kHistBins; i += kScoreCta) sm.hsh[i] = 0;
     __syncthreads();
+    griddep_wait();
 
     auto vis = [&](int t) { return min((a.q_pos[t] + 1) / a.m, a.max_blocks); };
 
@@ -546,6 +566,7 @@ __global__ void __launch_bounds__(kScoreCta, 2) index_score_kernel(ScoreArgs a) 
                     flag_status(a.status, kDevTimeout);
             }
         }
+        griddep_trigger();
         return;
     }
 
@@ -620,6 +641,7 @@ __global__ void __launch_bounds__(kScoreCta, 2) index_score_kernel(ScoreArgs a) 
         }
     }
     if (a.hist) leave_query(a, ct, contrib(ct), sm);
+    griddep_trigger();
 }
 
 // ---------------------------------------------------------------- collect
@@ -630,6 +652,7 @@ __global__ void __launch_bounds__(256) collect_kernel(const float* __restrict__ 
                                                       int m, int max_blocks, uint64_t* __restrict__ cand,
                                                       int64_t cand_cap, unsigned* __restrict__ cnt) {
     const int t = blockIdx.y;
+    griddep_wait();
     const int V = min((q_pos[t] + 1) / m, max_blocks);
     const int j0 = blockIdx.x * kCollectKeys;
     if (j0 >= V) return;
@@ -674,92 +697,135 @@ __global__ void __launch_bounds__(256) collect_kernel(const float* __restrict__ 
         }
         pos += __popc(bal[e]);
     }
+    griddep_trigger();
 }
 
 // ---------------------------------------------------------------- final
-// Exact selection and ordering of a query's candidate list (n ~ k plus one
-// histogram bin).  grid (kRankCtas, T), kRankThreads threads.  Every CTA
-// stages the whole list in shared memory, finds the exact k-th largest key
-// with a radix select, compacts the k selected keys, and ranks its share of
-// them: a selected key's output slot is the number of selected keys above it
-// (all keys are distinct).  Lists longer than kRankCap are selected from
-// global memory by CTA 0 alone.
-constexpr int kRankThreads = 256;
-constexpr int kRankCtas = 16;
-constexpr int kRankCap = 12288;       // candidates held in shared memory (96 KB)
-constexpr int kRankSplit = 4;         // threads per ranked key
+// Exact ordering of a query's candidate list (n ~ k plus one histogram bin),
+// one CTA per query.  All keys are distinct, so a key's output slot is its
+// rank (the number of keys above it); slots >= k are dropped.  Ranks come
+// from a counting pass: every key shares the bits above the highest bit in
+// which the largest and smallest key differ, so the 11 bits below that bit
+// are an order-preserving bucket number; a key's rank is the count of keys in
+// higher buckets plus the count of larger keys in its own bucket.
+constexpr int kRankThreads = 1024;
+constexpr int kRankCap = 8192;        // candidates ranked from shared memory
+constexpr int kRankBins = 2048;
 
 __device__ __forceinline__ void write_out(int* out_idx, float* out_score, int64_t pos, uint64_t x) {
     out_idx[pos] = cand_index(x);
     if (out_score) out_score[pos] = cand_score(x);
 }
 
+// Rank the n distinct nonzero keys v[0..n) (shared) and write those of rank
+// < k.  Scratch: bucket[n] (shared), hist/start[kRankBins] (shared).
+__device__ void rank_write(const uint64_t* v, int n, int k, uint64_t* bucket, unsigned* hist, unsigned* start,
+                           int* out_idx, float* out_score, int64_t out_off) {
+    __shared__ unsigned long long red[2];
+    __shared__ unsigned wsum[32];
+    const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        red[0] = 0ull;
+        red[1] = ~0ull;
+    }
+    for (int i = tid; i < kRankBins; i += nth) hist[i] = 0;
+    __syncthreads();
+    unsigned long long mx = 0ull, mn = ~0ull;
+    for (int i = tid; i < n; i += nth) {
+        mx = v[i] > mx ? v[i] : mx;
+        mn = v[i] < mn ? v[i] : mn;
+    }
+    atomicMax(&red[0], mx);
+    atomicMin(&red[1], mn);
+    __syncthreads();
+    const uint64_t diff = red[0] ^ red[1];
+    const int hb = diff ? 63 - __clzll((long long)diff) : 0;
+    const int sh = hb > 10 ? hb - 10 : 0;
+    for (int i = tid; i < n; i += nth) atomicAdd(&hist[(unsigned)(v[i] >> sh) & (kRankBins - 1)], 1u);
+    __syncthreads();
+    // start[b] = number of keys in buckets above b (exclusive scan from the top)
+    constexpr int per = kRankBins / kRankThreads;   // 2
+    unsigned c[per], tot = 0;
+#pragma unroll
+    for (int e = 0; e < per; ++e) {
+        c[e] = hist[kRankBins - 1 - (tid * per + e)];
+        tot += c[e];
+    }
+    unsigned incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    unsigned before = 0;
+    for (int w2 = 0; w2 < warp; ++w2) before += wsum[w2];
+    unsigned run = before + incl - tot;
+#pragma unroll
+    for (int e = 0; e < per; ++e) {
+        start[kRankBins - 1 - (tid * per + e)] = run;
+        run += c[e];
+    }
+    __syncthreads();
+    // place every key in its bucket (order inside a bucket is arbitrary)
+    for (int i = tid; i < kRankBins; i += nth) hist[i] = start[i];   // hist becomes the fill cursor
+    __syncthreads();
+    for (int i = tid; i < n; i += nth) {
+        const uint64_t x = v[i];
+        bucket[atomicAdd(&hist[(unsigned)(x >> sh) & (kRankBins - 1)], 1u)] = x;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += nth) {
+        const uint64_t x = bucket[i];
+        const unsigned b = (unsigned)(x >> sh) & (kRankBins - 1);
+        const unsigned lo = start[b], hi = hist[b];   // hist[b] ended at the bucket's end
+        unsigned rank = lo;
+        for (unsigned j = lo; j < hi; ++j) rank += bucket[j] > x;
+        if (rank < (unsigned)k) write_out(out_idx, out_score, out_off + rank, x);
+    }
+}
+
+// grid (T), kRankThreads threads.
 __global__ void __launch_bounds__(kRankThreads) rank_kernel(const uint64_t* __restrict__ cand, int64_t cand_cap,
                                                           const unsigned* __restrict__ cnt, int k,
                                                           int* __restrict__ out_idx, float* __restrict__ out_score) {
-    extern __shared__ __align__(16) uint64_t v[];   // [kRankCap] list, then [CSA k max] selected
-    __shared__ unsigned hist[256];
+    extern __shared__ __align__(16) uint64_t v[];   // [kRankCap] list, [kRankCap] buckets
+    uint64_t* bucket = v + kRankCap;
+    __shared__ unsigned hist[kRankBins];
+    __shared__ unsigned start[kRankBins];
     __shared__ int misc[8];
-    uint64_t* sel = v + kRankCap;
-    const int t = blockIdx.y, r = blockIdx.x;
+    const int t = blockIdx.x;
+    griddep_wait();
     const int n = (int)cnt[t];
     const uint64_t* src = cand + (int64_t)t * cand_cap;
-    if (r == 0)   // padding when fewer than k candidates exist
-        for (int i = n + threadIdx.x; i < k; i += blockDim.x) {
-            out_idx[(int64_t)t * k + i] = -1;
-            if (out_score) out_score[(int64_t)t * k + i] = __int_as_float(0x7fc00000);
-        }
-    const bool in_smem = n <= kRankCap;
-    if (!in_smem && r != 0) return;
-    if (in_smem) {
+    for (int i = n + threadIdx.x; i < k; i += blockDim.x) {   // padding when fewer than k candidates exist
+        out_idx[(int64_t)t * k + i] = -1;
+        if (out_score) out_score[(int64_t)t * k + i] = __int_as_float(0x7fc00000);
+    }
+    int ns = n;
+    if (n <= kRankCap) {
         // stage with cp.async (every 16-byte piece in flight); an odd last
         // element is zero-filled past the end
         for (int i = 2 * threadIdx.x; i < n; i += 2 * blockDim.x) cp_async16(v + i, src + i, i + 1 < n ? 16 : 8);
         cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
-    }
-    const uint64_t* list = in_smem ? v : src;
-    const uint64_t thr = block_select(list, n, k, hist, misc);
-    // order-preserving compaction: every CTA builds the same array
-    __shared__ unsigned wcnt[kRankThreads / 32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int ns = 0;
-    for (int base = 0; base < n; base += kRankThreads) {
-        const int i = base + threadIdx.x;
-        const uint64_t x = i < n ? list[i] : 0ull;
-        const bool take = x != 0ull && x >= thr;
-        const unsigned bal = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) wcnt[warp] = __popc(bal);
+    } else {
+        // long list (many scores share the threshold bin): cut it to exactly
+        // k keys with a radix select over global memory first
+        const uint64_t thr = block_select(src, n, k, hist, misc);
+        if (threadIdx.x == 0) misc[4] = 0;
         __syncthreads();
-        int off = ns, tot = 0;
-        for (int w2 = 0; w2 < kRankThreads / 32; ++w2) {
-            if (w2 < warp) off += wcnt[w2];
-            tot += wcnt[w2];
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint64_t x = __ldcg(src + i);
+            if (x != 0ull && x >= thr) v[atomicAdd(&misc[4], 1)] = x;
         }
-        if (take) sel[off + __popc(bal & ((1u << lane) - 1u))] = x;
-        ns += tot;
         __syncthreads();
+        ns = misc[4];
     }
-    // ns = min(k, n)
-    // this CTA's share of the selected keys (all of them when the list was long)
-    const int c0 = in_smem ? (int)((int64_t)ns * r / kRankCtas) : 0;
-    const int c1 = in_smem ? (int)((int64_t)ns * (r + 1) / kRankCtas) : ns;
-    for (int base = c0; base < c1; base += kRankThreads / kRankSplit) {
-        const int e = base + threadIdx.x / kRankSplit, part = threadIdx.x % kRankSplit;
-        const uint64_t x = e < c1 ? sel[e] : ~0ull;
-        int r0 = 0, r1 = 0;
-        int j = part;
-        for (; j + kRankSplit < ns; j += 2 * kRankSplit) {
-            r0 += sel[j] > x;
-            r1 += sel[j + kRankSplit] > x;
-        }
-        if (j < ns) r0 += sel[j] > x;
-        int rank = r0 + r1;
-#pragma unroll
-        for (int off = 1; off < kRankSplit; off <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, off);
-        if (part == 0 && e < c1) write_out(out_idx, out_score, (int64_t)t * k + rank, x);
-    }
+    rank_write(v, ns, k, bucket, hist, start, out_idx, out_score, (int64_t)t * k);
+    griddep_trigger();
 }
 
 // ---------------------------------------------------------------- host
@@ -793,14 +859,14 @@ static cudaError_t launch_score_t(const ScoreArgs& a, cudaStream_t stream) {
     const int64_t U = (int64_t)a.T * a.units_per_q;
     const int64_t grid = std::min<int64_t>(U, (int64_t)sm_count(dev) * occ);
     if (grid <= 0) return cudaSuccess;
-    kern<<<(unsigned)grid, kScoreCta, smem, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kScoreCta), smem, stream, a);
 }
 
 cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
                                const void* kidx, int fmt, const float* kscale, int64_t kstride_elems, int64_t sstride,
                                int m, int max_blocks, int k, float* scores, int64_t ld_scores, unsigned* hist,
-                               unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream, int* launches) {
+                               unsigned* cnt, unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream,
+                               int* launches) {
     ScoreArgs a;
     a.q = q;
     a.w = w;
@@ -824,6 +890,13 @@ cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq,
     a.units_per_q = (max_blocks + kUnit - 1) / kUnit;
     const int nt = Hi > 8 ? 2 : 1;
     cudaError_t e;
+    if (hist) {   // hist, cnt, done are contiguous: T * (kHistBins + 2) words
+        const int64_t words = (int64_t)T * (kHistBins + 2);
+        const int blocks = (int)std::min<int64_t>((words + 255) / 256, 1024);
+        e = launch_pdl(zero_state_kernel, dim3(blocks), dim3(256), 0, stream, hist, words);
+        if (e != cudaSuccess) return e;
+        *launches += 1;
+    }
     if (fmt == 0) e = nt == 1 ? launch_score_t<0, 1>(a, stream) : launch_score_t<0, 2>(a, stream);
     else e = nt == 1 ? launch_score_t<1, 1>(a, stream) : launch_score_t<1, 2>(a, stream);
     *launches += 1;
@@ -835,14 +908,14 @@ cudaError_t launch_index_select_tail(const float* scores, int64_t ld_scores, con
                                      unsigned* cnt, int* out_idx, float* out_score, cudaStream_t stream,
                                      int* launches) {
     dim3 g1((max_blocks + kCollectKeys - 1) / kCollectKeys, T);
-    collect_kernel<<<g1, 256, 0, stream>>>(scores, ld_scores, thr, q_pos, m, max_blocks, cand, cand_cap, cnt);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(collect_kernel, g1, dim3(256), 0, stream, scores, ld_scores, thr, q_pos, m, max_blocks,
+                               cand, cand_cap, cnt);
     if (e != cudaSuccess) return e;
-    const size_t rank_smem = (size_t)(kRankCap + k) * 8;
+    const size_t rank_smem = (size_t)2 * kRankCap * 8;
     e = cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem);
     if (e != cudaSuccess) return e;
-    rank_kernel<<<dim3(kRankCtas, T), kRankThreads, rank_smem, stream>>>(cand, cand_cap, cnt, k, out_idx, out_score);
-    e = cudaGetLastError();
+    e = launch_pdl(rank_kernel, dim3(T), dim3(kRankThreads), rank_smem, stream, (const uint64_t*)cand, cand_cap,
+                   (const unsigned*)cnt, k, out_idx, out_score);
     if (e != cudaSuccess) return e;
     *launches += 2;
     return e;

@@ -86,7 +86,8 @@ def test_attend_validation(L):
     assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 16, 128, 0.1, f, NULL, f, 1000, NULL) == 4
     h = L.hca_attend
     assert h(f, f, f, 2, 64, f, 0, f, 0, 128, -1, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 2
-    assert csa.csa_attend_workspace_size(8, 64, 1152) >= 8 * 9 * 64 * 130 * 4
+    assert csa.csa_attend_workspace_size(8, 64, 1152) >= 256
+    assert csa.hca_attend_workspace_size(16, 64, 8320) >= 16 * 17 * 64 * 130 * 4
 
 
 def test_library_calls_no_allocator():
