@@ -36,8 +36,10 @@ sys.path.insert(0, ROOT)
 from long_context_sparse_03_b200 import workloads as wl  # noqa: E402
 
 WORKLOADS = {"csa_decode_1m": wl.CSA_DECODE_1M, "csa_decode_64k": wl.CSA_DECODE_64K_RAGGED,
-             "csa_decode_4k": wl.CSA_DECODE_4K, "hca_decode_1m": wl.HCA_DECODE_1M}
+             "csa_decode_4k": wl.CSA_DECODE_4K, "hca_decode_1m": wl.HCA_DECODE_1M,
+             "csa_prefill_8k": wl.CSA_PREFILL_8K}
 METRIC = "CSA decode tokens/s and achieved HBM GB/s at 1M context, 1xB200"
+METRIC_PREFILL = "CSA chunked-prefill tokens/s and indexer tensor TFLOP/s, 1xB200"
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -128,6 +130,17 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor peak (burst: the kernel is timed alone)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def measured_hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -210,14 +223,15 @@ def main():
         return run_reference(args, w, rank, world, dev)
 
     from long_context_sparse_03_b200 import csa
-    from long_context_sparse_03_b200.decode import CsaDecoder, HcaDecoder
+    from long_context_sparse_03_b200.decode import CsaDecoder, CsaPrefill, HcaDecoder
     csa.lib()
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
     inp = wl.make_inputs(w, device=str(dev))
     hca = w.kind == "hca_decode"
+    prefill = w.kind == "csa_prefill"
     fmt = csa.FMT_BF16 if args.kidx == "bf16" else csa.FMT_FP8E4M3
-    dec = HcaDecoder(inp) if hca else CsaDecoder(inp, fmt)
+    dec = HcaDecoder(inp) if hca else (CsaPrefill(inp) if prefill else CsaDecoder(inp, fmt))
 
     def evpair():
         return (torch.cuda.Event(enable_timing=True, external=True),
@@ -244,7 +258,7 @@ def main():
     K = args.steps
 
     # host-side buffers of the end-to-end path
-    e2e_on = not hca
+    e2e_on = not hca and not prefill
     if e2e_on:
         pos = inp.lens.long() - 1
         bidx = torch.arange(w.B, device=dev)
@@ -291,20 +305,30 @@ def main():
     ms_per_step = total_ms_max / K
     tokens = reduce_sum(dec.T * K, dev)
     value = tokens / (total_ms_max / 1e3)
-    ab = dec.algorithmic_bytes()
-    step_gbs = ab["total"] / (ms_per_step / 1e3) / 1e9
-
-    # dominant kernel: the indexer scoring stream (CSA) or the attention (HCA)
-    peak, peak_src = measured_hbm_peak()
     k_ms = float(np.mean([a.elapsed_time(b) for a, b in evk]))
-    if hca:
-        kbytes, kname = ab["total"], "attend_kernel+combine_kernel"
+    if prefill:
+        fl = dec.flops()
+        ab = {"total": None}
+        step_gbs = None
+        tf_peak, tf_src = measured_tensor_peak()
+        ach = fl["indexer"] / (k_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": "index_score_kernel", "achieved": round(ach, 2), "peak": tf_peak,
+                "unit": "TFLOP/s", "frac": round(ach / tf_peak, 4), "peak_source": tf_src, "traffic": None,
+                "algorithmic_flops_per_launch": fl["indexer"], "avg_launch_ms": round(k_ms, 5),
+                "step_flops": fl}
     else:
-        kbytes, kname = ab["keys"], "index_score_kernel"
-    ach = kbytes / (k_ms / 1e3) / 1e9
-    roof = {"bound": "hbm", "kernel": kname, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(ach / peak, 4), "peak_source": peak_src, "traffic": None,
-            "algorithmic_bytes_per_launch": kbytes, "avg_launch_ms": round(k_ms, 5)}
+        ab = dec.algorithmic_bytes()
+        step_gbs = ab["total"] / (ms_per_step / 1e3) / 1e9
+        # dominant kernel: the indexer scoring stream (CSA) or the attention (HCA)
+        peak, peak_src = measured_hbm_peak()
+        if hca:
+            kbytes, kname = ab["total"], "attend_kernel+combine_kernel"
+        else:
+            kbytes, kname = ab["keys"], "index_score_kernel"
+        ach = kbytes / (k_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": kname, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "peak_source": peak_src, "traffic": None,
+                "algorithmic_bytes_per_launch": kbytes, "avg_launch_ms": round(k_ms, 5)}
 
     # end to end through the public API with pinned host buffers
     e2e = None
@@ -331,7 +355,7 @@ def main():
 
     # CPU baseline: the oracle on this workload's host cores (rank 0, N = 1)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not prefill:
         d = oracle_inputs(inp, w)
         done, dt = time_oracle(d, w, steps=max(1, args.steps), budget_s=20.0)
         cpu = {"value": round(done * dec.T / dt, 3), "unit": "tokens/s", "cores": d["o"].num_threads(),
@@ -341,7 +365,7 @@ def main():
 
     if rank == 0:
         rec = {
-            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC_PREFILL if prefill else METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if fmt == 0 else "bf16+e4m3",
             "data": "synthetic (seeded N(0,1), weights 1/sqrt(fan_in)); caches resident in HBM",
@@ -350,7 +374,7 @@ def main():
                        "indexer_keys": args.kidx, "l2": "inputs larger than L2 (268 MB of keys per step); plus a 256 MiB write then read before every step",
                        "parallelism": f"replicas x{world} (independent batches per GPU)",
                        "timing": "K steps captured in one CUDA graph, CUDA events inside it"},
-            "step_hbm_gbs": round(step_gbs, 1), "step_algorithmic_bytes": ab["total"],
+            "step_hbm_gbs": None if step_gbs is None else round(step_gbs, 1), "step_algorithmic_bytes": ab["total"],
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "clocks": clk.summary(),
             "cache_build": {"ms": round(build_ms, 3), "raw_bytes_read": raw_bytes,

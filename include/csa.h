@@ -98,6 +98,7 @@ enum { CSA_DEV_BAD_INDEX = 1u, CSA_DEV_TIMEOUT = 2u };
 #define CSA_MAX_K 2048     /* top-k: 1..2048 */
 #define CSA_MAX_W 1024     /* window: 0..1024 */
 #define CSA_MAX_D 7168     /* indexer d_model and rank: multiples of 8 up to this */
+#define CSA_MAX_T 65535    /* queries per call (T) and sequences per compress call (B) */
 /* attention heads H: 16, 32, 48, ..., 128 (a multiple of 16) */
 
 /* Human-readable name of a status code (static string). */
@@ -142,8 +143,13 @@ CSA_API csa_status csa_status_check(void* ws, size_t ws_bytes, csa_stream_t stre
  * out_scale  fp32 [B][scale_seq_stride] for E4M3 (NULL for bf16): s_j = amax_j/448
  *            of the bf16-rounded row (1 if the row is all zeros), codes =
  *            e4m3_rn_satfinite(x / s_j) in fp32.
- * Accumulation: fp32, one FMA per position in order i = 0..m-1; bf16 output
- * rounded to nearest even.  Blocks outside the range are not written.
+ * B          0..CSA_MAX_T sequences.
+ * The grid is bounded by what the SMs hold at once (each CTA loops over its
+ * rows), so a blk_hi far past the longest sequence costs nothing.
+ * Accumulation: fp32; for m < 16 one FMA chain over i = 0..m-1, for m >= 16
+ * sixteen (d = 128) or thirty-two (d = 64) interleaved chains added in a
+ * fixed order; bf16 output rounded to nearest even.  Blocks outside the
+ * range are not written.
  */
 CSA_API csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* lens,
                         int B, int d, int m, const float* pool_logits,
@@ -248,7 +254,7 @@ CSA_API size_t hca_attend_workspace_size(int T, int H, int max_rows);
  * lse fp32 [T][H] (natural log of the softmax denominator, -inf for an
  * empty set) or NULL.  An empty attended set gives out = 0.
  * fp32 logits, softmax and accumulation; split-K over fixed 64-row splits
- * (512-row for hca_attend) merged in a fixed order.
+ * (256-row for hca_attend) merged in a fixed order.
  */
 CSA_API csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
                              int T, int H, const void* comp, int64_t comp_seq_stride,

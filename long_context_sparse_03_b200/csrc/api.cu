@@ -121,6 +121,7 @@ csa_status check_index_common(const float* q, const float* w, const int32_t* q_s
                               int Hi, const void* kidx, int kidx_fmt, const float* kidx_scale,
                               int64_t kidx_seq_stride, int64_t scale_seq_stride, int m, int max_blocks) {
     REQUIRE(T >= 0, CSA_ERR_SHAPE, "T = %d < 0", T);
+    REQUIRE(T <= CSA_MAX_T, CSA_ERR_UNSUPPORTED, "T = %d > %d", T, CSA_MAX_T);
     REQUIRE(Hi >= 1 && Hi <= CSA_MAX_HI, CSA_ERR_UNSUPPORTED, "Hi = %d outside 1..%d", Hi, CSA_MAX_HI);
     REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
     REQUIRE(max_blocks >= 1, CSA_ERR_SHAPE, "max_blocks = %d < 1", max_blocks);
@@ -185,6 +186,7 @@ csa_status csa_compress(const void* raw, int64_t raw_seq_stride, const int32_t* 
                         const float* pool_logits, int blk_lo, int blk_hi, void* out, int64_t out_seq_stride,
                         int out_fmt, float* out_scale, int64_t scale_seq_stride, csa_stream_t stream) {
     REQUIRE(B >= 0, CSA_ERR_SHAPE, "B = %d < 0", B);
+    REQUIRE(B <= CSA_MAX_T, CSA_ERR_UNSUPPORTED, "B = %d > %d", B, CSA_MAX_T);
     REQUIRE(d == 64 || d == 128, CSA_ERR_UNSUPPORTED, "d = %d (64 or 128)", d);
     REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
     REQUIRE(out_fmt == CSA_FMT_BF16 || (out_fmt == CSA_FMT_FP8E4M3 && d == 64), CSA_ERR_UNSUPPORTED,
@@ -312,6 +314,7 @@ csa_status csa_index_stage_score(const float* q, const float* w, const int32_t* 
 csa_status csa_index_stage_merge(const int32_t* q_pos, int T, int m, int max_blocks, int k, int32_t* out_idx,
                                  float* out_score, void* ws, size_t ws_bytes, csa_stream_t stream) {
     REQUIRE(T >= 0 && max_blocks >= 1, CSA_ERR_SHAPE, "T = %d, max_blocks = %d", T, max_blocks);
+    REQUIRE(T <= CSA_MAX_T, CSA_ERR_UNSUPPORTED, "T = %d > %d", T, CSA_MAX_T);
     REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
     REQUIRE(k >= 1 && k <= CSA_MAX_K, CSA_ERR_UNSUPPORTED, "k = %d outside 1..%d", k, CSA_MAX_K);
     if (T == 0) return ok();
@@ -340,6 +343,7 @@ csa_status csa_index_topk(const void* h, int D, int r, const void* W_dq, const v
                           int max_blocks, int k, int32_t* out_idx, float* out_score, void* ws, size_t ws_bytes,
                           csa_stream_t stream) {
     REQUIRE(T >= 0, CSA_ERR_SHAPE, "T = %d < 0", T);
+    REQUIRE(T <= CSA_MAX_T, CSA_ERR_UNSUPPORTED, "T = %d > %d", T, CSA_MAX_T);
     REQUIRE(Hi >= 1 && Hi <= CSA_MAX_HI, CSA_ERR_UNSUPPORTED, "Hi = %d outside 1..%d", Hi, CSA_MAX_HI);
     REQUIRE(r >= 0, CSA_ERR_SHAPE, "r = %d < 0", r);
     REQUIRE(k >= 1 && k <= CSA_MAX_K, CSA_ERR_UNSUPPORTED, "k = %d outside 1..%d", k, CSA_MAX_K);
@@ -380,6 +384,7 @@ static csa_status attend_common(const char* who, const void* q, const int32_t* q
                                 float scale, void* out, float* lse, void* ws, size_t ws_bytes,
                                 csa_stream_t stream) {
     REQUIRE(T >= 0, CSA_ERR_SHAPE, "T = %d < 0", T);
+    REQUIRE(T <= CSA_MAX_T, CSA_ERR_UNSUPPORTED, "T = %d > %d", T, CSA_MAX_T);
     REQUIRE(H >= 16 && H <= 128 && H % 16 == 0, CSA_ERR_UNSUPPORTED, "H = %d (16..128, multiple of 16)", H);
     REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
     REQUIRE(W >= 0 && W <= CSA_MAX_W, CSA_ERR_UNSUPPORTED, "W = %d outside 0..%d", W, CSA_MAX_W);
@@ -464,6 +469,7 @@ csa_status csa_sparse_attend_noalloc(const void* q, const int32_t* q_seq, const 
                                      void* out, float* lse, csa_stream_t stream) {
     REQUIRE(k >= 1 && k <= CSA_MAX_K, CSA_ERR_UNSUPPORTED, "k = %d outside 1..%d", k, CSA_MAX_K);
     REQUIRE(T >= 0, CSA_ERR_SHAPE, "T = %d < 0", T);
+    REQUIRE(T <= CSA_MAX_T, CSA_ERR_UNSUPPORTED, "T = %d > %d", T, CSA_MAX_T);
     REQUIRE(H >= 16 && H <= 128 && H % 16 == 0, CSA_ERR_UNSUPPORTED, "H = %d (16..128, multiple of 16)", H);
     REQUIRE(m >= 1 && m <= CSA_MAX_M, CSA_ERR_UNSUPPORTED, "m = %d outside 1..%d", m, CSA_MAX_M);
     REQUIRE(W >= 0 && W <= CSA_MAX_W, CSA_ERR_UNSUPPORTED, "W = %d outside 0..%d", W, CSA_MAX_W);

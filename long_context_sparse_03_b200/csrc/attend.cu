@@ -21,7 +21,7 @@
 namespace csa {
 
 constexpr int kCsaRowsPerSplit = 64;    // CSA: k + W rows per query, latency-bound
-constexpr int kHcaRowsPerSplit = 512;   // HCA: thousands of rows per query
+constexpr int kHcaRowsPerSplit = 256;   // HCA: thousands of rows per query
 constexpr int kRowBlock = 64;
 constexpr int kRowStride = 136;  // bf16 per smem row (272 B: conflict-free ldmatrix)
 

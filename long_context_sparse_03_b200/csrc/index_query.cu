@@ -247,12 +247,28 @@ static cudaError_t launch_gemv(const bf16* W0, int n0, float* Y0, int ld0, const
                       Y0, ld0, W1, n1, Y1, ld1, K, X, T);
 }
 
+template <typename AT>
+cudaError_t launch_gemm_tn(const AT* A, int M, int K, const bf16* B0, int n0, float* C0, int ldc0, const bf16* B1,
+                           int n1, float* C1, int ldc1, cudaStream_t stream);
+
+// Many queries (chunked prefill): the projections are tiled GEMMs.
+constexpr int kGemmMinT = 64;
+
 // q_out [T][Hi*64], w_out [T][Hi], u_ws [T][r] (fp32 scratch).
 cudaError_t launch_index_query(const void* h, int T, int D, int r, int Hi, const void* W_dq, const void* W_uq,
                                const void* W_w, float* q_out, float* w_out, float* u_ws, cudaStream_t stream,
                                int* launches) {
     const bf16* hb = reinterpret_cast<const bf16*>(h);
     cudaError_t e;
+    if (T >= kGemmMinT && D % 32 == 0 && r % 32 == 0) {
+        e = launch_gemm_tn<bf16>(hb, T, D, reinterpret_cast<const bf16*>(W_dq), r, u_ws, r,
+                                 reinterpret_cast<const bf16*>(W_w), Hi, w_out, Hi, stream);
+        if (e != cudaSuccess) return e;
+        e = launch_gemm_tn<float>(u_ws, T, r, reinterpret_cast<const bf16*>(W_uq), Hi * 64, q_out, Hi * 64, nullptr, 0,
+                                  nullptr, 0, stream);
+        *launches += 2;
+        return e;
+    }
     if (D % (64 * kMmaWarps) == 0) {
         const size_t smem = (size_t)kGemvTT * D * 2 + (size_t)kMmaWarps * 128 * 4;
         e = cudaFuncSetAttribute(gemv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

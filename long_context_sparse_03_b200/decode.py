@@ -170,3 +170,69 @@ class HcaDecoder:
         rows = int(vis.sum().item()) * 256
         window = int(self.inp.lens.long().clamp(max=w.W).sum().item()) * 256
         return {"compressed": rows, "window": window, "total": rows + window}
+
+
+class CsaPrefill:
+    """Chunked causal CSA prefill: T new tokens appended after a context whose
+    compressed caches already exist.  One step compresses the new complete
+    blocks, projects the indexer queries of all T tokens, selects each
+    token's top-k visible blocks and attends over them plus the window."""
+
+    def __init__(self, inp: Inputs, stream: torch.cuda.Stream | None = None):
+        w = inp.w
+        self.inp, self.w = inp, w
+        self.stream = stream
+        dev = inp.raw_kv.device
+        self.T = inp.T
+        self.N = w.max_blocks
+        self.n_old = (w.L - w.T_new) // w.m      # blocks that exist before the chunk
+        self.scale = csa.softmax_scale(128)
+        self.comp = torch.empty((w.B, self.N, 128), dtype=torch.bfloat16, device=dev)
+        self.kidx = torch.empty((w.B, self.N, 64), dtype=torch.bfloat16, device=dev)
+        self.q_idx = torch.empty((self.T, w.Hi, 64), dtype=torch.float32, device=dev)
+        self.w_idx = torch.empty((self.T, w.Hi), dtype=torch.float32, device=dev)
+        self.idx = torch.empty((self.T, w.k), dtype=torch.int32, device=dev)
+        self.idx_score = torch.empty((self.T, w.k), dtype=torch.float32, device=dev)
+        self.out = torch.empty((self.T, w.H, 128), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.T, w.H), dtype=torch.float32, device=dev)
+        self.ws_idx = csa.Workspace(csa.csa_index_workspace_size(self.T, w.r, w.Hi, w.k, self.N), dev, self.stream)
+        self.ws_att = csa.Workspace(csa.csa_attend_workspace_size(self.T, w.H, w.k + w.W), dev, self.stream)
+
+    def _s(self):
+        return self.stream or torch.cuda.current_stream()
+
+    def build_caches(self):
+        """Compress the context that precedes the chunk."""
+        i, w = self.inp, self.w
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, 0, self.n_old, self.comp, stream=self.stream)
+        csa.csa_compress(i.raw_ki, i.lens, i.z_ki, w.m, 0, self.n_old, self.kidx, stream=self.stream)
+
+    def step(self, ev_score: tuple | None = None):
+        i, w = self.inp, self.w
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, self.n_old, self.N, self.comp, stream=self.stream)
+        csa.csa_compress(i.raw_ki, i.lens, i.z_ki, w.m, self.n_old, self.N, self.kidx, stream=self.stream)
+        csa.csa_index_query(i.h, i.W_dq, i.W_uq, i.W_w, self.q_idx, self.w_idx, self.ws_idx, stream=self.stream)
+        if ev_score:
+            ev_score[0].record(self._s())
+        csa.csa_index_stage_score(self.q_idx, self.w_idx, i.q_seq, i.q_pos, self.kidx, w.m, self.N, w.k, self.ws_idx,
+                                  stream=self.stream)
+        if ev_score:
+            ev_score[1].record(self._s())
+        csa.csa_index_stage_merge(i.q_pos, w.m, self.N, w.k, self.idx, self.idx_score, self.ws_idx, stream=self.stream)
+        csa.csa_sparse_attend(i.q, i.q_seq, i.q_pos, self.comp, i.raw_kv, w.m, self.idx, w.W, self.scale, self.out,
+                              self.lse, self.ws_att, stream=self.stream)
+        return self.out
+
+    def flops(self) -> dict:
+        """Dense-equivalent work of the step: the indexer contraction over the
+        visible blocks, the projections and the attention (multiply-add = 2)."""
+        w = self.w
+        pos = self.inp.q_pos.long()
+        vis = ((pos + 1) // w.m).clamp(max=self.N).sum().item()
+        win = (pos + 1).clamp(max=w.W).sum().item()
+        sel = ((pos + 1) // w.m).clamp(max=w.k).sum().item()
+        T = self.T
+        idx = 2 * vis * w.Hi * 64
+        proj = 2 * T * (w.D * (w.r + w.Hi) + w.r * w.Hi * 64)
+        att = 2 * 2 * (sel + win) * w.H * 128
+        return {"indexer": int(idx), "projection": int(proj), "attention": int(att), "total": int(idx + proj + att)}

@@ -50,6 +50,7 @@ def test_compress_validation(L):
     assert s(_fake(), 0, _fake(), 1, 128, 4, _fake(), -2, 4, _fake(), 0, 0, NULL, 0, NULL) == 2
     assert s(_fake(0x10004), 0, _fake(), 1, 128, 4, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 8
     assert s(_fake(), 12, _fake(), 1, 128, 4, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 8
+    assert s(_fake(), 0, _fake(), 70000, 128, 4, _fake(), 0, 4, _fake(), 0, 0, NULL, 0, NULL) == 3  # B > 65535
     # empty work is a no-op success, even with NULL pointers
     assert s(NULL, 0, NULL, 0, 128, 4, NULL, 0, 4, NULL, 0, 0, NULL, 0, NULL) == 0
     assert s(NULL, 0, NULL, 3, 128, 4, NULL, 2, 2, NULL, 0, 0, NULL, 0, NULL) == 0
@@ -67,6 +68,7 @@ def test_index_validation(L):
     assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 4, 100, 16, f, NULL, f, 300, NULL) == 4
     assert sel(f, f, f, f, 2, 8, f, 0, NULL, 0, 0, 4, 100, 16, NULL, NULL, f, 1 << 20, NULL) == 1
     assert sel(f, f, f, f, 2, 8, f, 0, NULL, 12, 0, 4, 100, 16, f, NULL, f, 1 << 20, NULL) == 8
+    assert sel(f, f, f, f, 70000, 8, f, 0, NULL, 0, 0, 4, 100, 16, f, NULL, f, 1 << 40, NULL) == 3  # T > 65535
     need = csa.csa_index_workspace_size(2, 512, 8, 16, 100)
     assert need > 256
     q = L.csa_index_query
@@ -84,6 +86,7 @@ def test_attend_validation(L):
     assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 0, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 3
     assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 16, 128, float("inf"), f, NULL, f, 1 << 24, NULL) == 2
     assert a(f, f, f, 2, 64, f, 0, f, 0, 4, f, 16, 128, 0.1, f, NULL, f, 1000, NULL) == 4
+    assert a(f, f, f, 65536, 64, f, 0, f, 0, 4, f, 16, 128, 0.1, f, NULL, f, 1 << 40, NULL) == 3  # T > 65535
     h = L.hca_attend
     assert h(f, f, f, 2, 64, f, 0, f, 0, 128, -1, 128, 0.1, f, NULL, f, 1 << 24, NULL) == 2
     assert csa.csa_attend_workspace_size(8, 64, 1152) >= 256

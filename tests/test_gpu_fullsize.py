@@ -181,3 +181,66 @@ def test_hca_decode_1m_b16(oracle):
                         ro, rl)
     del inp, comp
     torch.cuda.empty_cache()
+
+
+def test_csa_prefill_8k_sampled(oracle):
+    """Chunked prefill (8192 tokens after 131072): the whole chunk runs in one
+    launch configuration; 12 queries spread over the chunk are judged."""
+    from long_context_sparse_03_b200.decode import CsaPrefill
+    w = wl.CSA_PREFILL_8K
+    inp = wl.make_inputs(w, device="cuda")
+    pf = CsaPrefill(inp)
+    pf.build_caches()
+    i = inp
+    N, T, m = w.max_blocks, w.T_new, w.m
+    csa.csa_compress(i.raw_kv, i.lens, i.z_kv, m, pf.n_old, N, pf.comp)
+    csa.csa_compress(i.raw_ki, i.lens, i.z_ki, m, pf.n_old, N, pf.kidx)
+    torch.cuda.synchronize()
+    lens = i.lens.cpu().numpy()
+    raw_kv, raw_ki = _bits(i.raw_kv), _bits(i.raw_ki)
+    ck, _ = oracle.compress(raw_kv, lens, i.z_kv.cpu().numpy(), 0, 1 << 30)
+    kk, _ = oracle.compress(raw_ki, lens, i.z_ki.cpu().numpy(), 0, 1 << 30)
+    a = oracle.pool_weights(i.z_kv.cpu().numpy())
+    x = bf16_bits_to_f64(raw_kv[0, :N * m]).reshape(N, m, 128)[pf.n_old:]
+    check_compress_bf16(_bits(pf.comp[0, pf.n_old:N]), ck[0, pf.n_old:N],
+                        absum=np.einsum("jid,id->jd", np.abs(x), np.abs(a)), m=m)
+    pf.comp[0, :N] = _to_dev(ck[0, :N])
+    pf.kidx[0, :N] = _to_dev(kk[0, :N])
+    # projection of all T queries on the GPU (GEMM path) vs the oracle on samples
+    csa.csa_index_query(i.h, i.W_dq, i.W_uq, i.W_w, pf.q_idx, pf.w_idx, pf.ws_idx)
+    sample = np.linspace(0, T - 1, 12).astype(int)
+    h = _bits(i.h)[sample]
+    rq, rw = oracle.index_query(h, _bits(i.W_dq), _bits(i.W_uq), _bits(i.W_w))
+    gq = pf.q_idx[torch.from_numpy(sample).cuda()].cpu().numpy().astype(np.float64)
+    gw = pf.w_idx[torch.from_numpy(sample).cuda()].cpu().numpy().astype(np.float64)
+    for t in range(len(sample)):
+        assert np.abs(gq[t] - rq[t]).max() <= 1e-5 * np.abs(rq[t]).max()
+        assert np.abs(gw[t] - rw[t]).max() <= 1e-5 * np.abs(rw[t]).max()
+    # selection over all T queries, the sampled ones driven by the oracle's q, w
+    q32, w32 = rq.astype(np.float32), rw.astype(np.float32)
+    st = torch.from_numpy(sample).cuda()
+    pf.q_idx[st] = torch.from_numpy(q32).cuda()
+    pf.w_idx[st] = torch.from_numpy(w32).cuda()
+    csa.csa_index_select(pf.q_idx, pf.w_idx, i.q_seq, i.q_pos, pf.kidx, m, N, w.k, pf.idx, pf.idx_score, pf.ws_idx)
+    pf.ws_idx.check()
+    q_pos = i.q_pos.cpu().numpy()[sample]
+    S = oracle.index_scores(q32.astype(np.float64), w32.astype(np.float64), np.zeros(len(sample), np.int32), q_pos,
+                            kk, m, N)
+    oi, _ = oracle.topk(S, q_pos, m, w.k)
+    gi, gs = pf.idx[st].cpu().numpy(), pf.idx_score[st].cpu().numpy()
+    kf = bf16_bits_to_f64(kk[0])
+    for t in range(len(sample)):
+        A = score_scale(q32[t].astype(np.float64), w32[t].astype(np.float64), kf)
+        V = min((int(q_pos[t]) + 1) // m, N)
+        check_topk(gi[t], gs[t], S[t], A, V, w.k)
+    # attention over the oracle's selection (whole chunk in one call)
+    idx_all = pf.idx.clone()
+    idx_all[st] = torch.from_numpy(oi).cuda()
+    csa.csa_sparse_attend(i.q, i.q_seq, i.q_pos, pf.comp, i.raw_kv, m, idx_all, w.W, 128 ** -0.5, pf.out, pf.lse,
+                          pf.ws_att)
+    pf.ws_att.check()
+    qa = _bits(i.q)[sample]
+    ro, rl = oracle.sparse_attend(qa, np.zeros(len(sample), np.int32), q_pos, ck, raw_kv, m, oi, w.W, 128 ** -0.5)
+    check_attention(bf16_bits_to_f64(host_bits(pf.out[st])), pf.lse[st].cpu().numpy().astype(np.float64), ro, rl)
+    del inp, pf
+    torch.cuda.empty_cache()

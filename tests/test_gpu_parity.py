@@ -114,7 +114,8 @@ def test_compress_relative_range(oracle):
 
 
 # ---------------------------------------------------------------- indexer
-@pytest.mark.parametrize("T,D,r,Hi", [(1, 1024, 256, 4), (8, 4096, 512, 8), (5, 512, 64, 16), (33, 256, 32, 3)])
+@pytest.mark.parametrize("T,D,r,Hi", [(1, 1024, 256, 4), (8, 4096, 512, 8), (5, 512, 64, 16), (33, 256, 32, 3),
+                                      (200, 1024, 256, 8), (130, 4096, 512, 8), (64, 512, 64, 16), (77, 96, 40, 5)])
 def test_index_query(oracle, T, D, r, Hi):
     rng = np.random.default_rng(T + D + Hi)
     h = rand_bf16(rng, (T, D))
