@@ -82,17 +82,42 @@ class CsaDecoder:
     def _s(self):
         return self.stream or torch.cuda.current_stream()
 
+    def _side_streams(self):
+        if not hasattr(self, "_side"):
+            dev = self.inp.raw_kv.device
+            self._side = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+            self._ev = [torch.cuda.Event() for _ in range(3)]
+        return self._side
+
     def step(self, ev_score: tuple | None = None):
         """One decode step on device-resident inputs.  ev_score: optional
-        (start, end) CUDA events recorded around the scoring kernel."""
-        self.refresh()
+        (start, end) CUDA events recorded around the scoring kernel.
+
+        The two refreshes are independent of the indexer query, so they run
+        on side streams: the key refresh beside the query projection (joined
+        before scoring), the latent refresh beside the whole indexer (joined
+        before attention).  Inside a captured graph these become parallel
+        branches."""
+        i, w = self.inp, self.w
+        main = self._s()
+        side_kv, side_ki = self._side_streams()
+        ev_fork, ev_ki, ev_kv = self._ev
+        ev_fork.record(main)
+        side_kv.wait_event(ev_fork)
+        side_ki.wait_event(ev_fork)
+        csa.csa_compress(i.raw_kv, i.lens, i.z_kv, w.m, -1, 1, self.comp, stream=side_kv)
+        ev_kv.record(side_kv)
+        csa.csa_compress(i.raw_ki, i.lens, i.z_ki, w.m, -1, 1, self.kidx, self.fmt, self.kscale, stream=side_ki)
+        ev_ki.record(side_ki)
         self.query()
+        main.wait_event(ev_ki)
         if ev_score:
-            ev_score[0].record(self._s())
+            ev_score[0].record(main)
         self.score()
         if ev_score:
-            ev_score[1].record(self._s())
+            ev_score[1].record(main)
         self.merge()
+        main.wait_event(ev_kv)
         self.attend()
         return self.out
 
