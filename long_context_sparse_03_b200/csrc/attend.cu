@@ -12,10 +12,15 @@
 // 64-row blocks gathered into shared memory with cp.async (the next block is
 // in flight while this one computes), an online softmax in registers, then
 // O += P V with P re-packed from the S accumulators.  The attended row list
-// of a query is cut into fixed splits (64 rows for CSA, 512 for HCA; never a
-// function of the batch, so results are batch invariant); each CTA writes
-// its split's (max, sum, unnormalised output) and a combine kernel merges
-// the splits in order.
+// of a query is cut into fixed splits (64 rows for CSA, 256 for HCA; never a
+// function of the batch).  Each split yields (max, sum, unnormalised output)
+// from a fresh online softmax, and the splits are folded in split order with
+// one fixed formula (fold_split).  Two launch shapes compute exactly the same
+// thing: with few queries one CTA per (split, query) writes its partial and a
+// combine kernel folds them; with many queries one CTA per query walks its
+// splits in order and folds them in registers (no partials, no combine
+// launch).  Both use the same per-split code and the same fold, so a
+// query's output is bit-identical whichever shape runs: batch invariant.
 #include "common.cuh"
 
 namespace csa {
@@ -67,30 +72,53 @@ __device__ __forceinline__ const bf16* row_ptr(const AttnArgs& a, int t, int b, 
     return a.raw + (int64_t)b * a.raw_stride + (int64_t)s * 128;
 }
 
-template <int NW>
-__global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
+// Fold split partial (mi, li, oi) into the running (M, L, O):
+// M' = max(M, mi), a = 2^(M - M'), b = 2^(mi - M') (0 for an empty side),
+// L = L a + li b, O = O a + oi b.  An empty split (mi = -inf, li = 0, oi = 0)
+// leaves the running state exactly unchanged.
+__device__ __forceinline__ void fold_scales(float M, float mi, float& Mn, float& fa, float& fb) {
+    Mn = fmaxf(M, mi);
+    fa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+    fb = mi == -INFINITY ? 0.f : exp2f(mi - Mn);
+}
+__device__ __forceinline__ float fold_val(float X, float fa, float xi, float fb) { return fmaf(X, fa, xi * fb); }
+
+// Final normalisation shared by both launch shapes.
+__device__ __forceinline__ float fin_out(float O, float L) { return L > 0.f ? O / L : 0.f; }
+__device__ __forceinline__ float fin_lse(float M, float L) {
+    return L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+// One CTA: NW warps x 16 heads of query t (blockIdx.y, or blockIdx.x when
+// FUSED).  Split shape: the row blocks of split blockIdx.x, partial to
+// part_o / part_ml.  FUSED: every split of the query in order, folded in
+// registers, output written directly.  The row blocks of consecutive splits
+// form one sequence, so the gather of the next block (cp.async, double
+// buffered) overlaps the current one across split boundaries too.
+template <int NW, bool FUSED>
+__global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a, bf16* __restrict__ out, float* __restrict__ lse) {
     constexpr int H = NW * 16;
     __shared__ __align__(16) bf16 rows_sh[2][kRowBlock * kRowStride];
     __shared__ int valid_sh[2][kRowBlock];
 
-    const int t = blockIdx.y, sp = blockIdx.x;
+    const int t = FUSED ? blockIdx.x : blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
     griddep_wait();
     const int b = a.q_seq[t], p = a.q_pos[t];
     const int V = a.idx ? (p + 1) / a.m : min((p + 1) / a.m, a.max_blocks);
     const int nsel = a.idx ? a.k : V;
     const int total = nsel + a.W;
-    const int pos0 = sp * a.rows_per_split;
-    const int npos = max(0, min(a.rows_per_split, total - pos0));
-    const int nblk = (npos + kRowBlock - 1) / kRowBlock;
+    const int bps = a.rows_per_split / kRowBlock;          // row blocks per split
+    const int nb_total = (total + kRowBlock - 1) / kRowBlock;
+    const int gb_lo = FUSED ? 0 : blockIdx.x * bps;
+    const int gb_hi = FUSED ? nb_total : min(nb_total, gb_lo + bps);
 
-    // issue the gather of row block `blk` into buffer `buf`
-    auto gather = [&](int blk, int buf) {
+    // issue the gather of row block `gb` (list positions gb*64 ..) into buffer `buf`
+    auto gather = [&](int gb, int buf) {
         for (int i = threadIdx.x; i < kRowBlock * 16; i += NW * 32) {
             const int r = i >> 4, c = i & 15;
-            const int pos = pos0 + blk * kRowBlock + r;
-            const bf16* src = nullptr;
-            if (blk * kRowBlock + r < npos) src = row_ptr(a, t, b, p, V, nsel, pos);
+            const int pos = gb * kRowBlock + r;
+            const bf16* src = pos < total ? row_ptr(a, t, b, p, V, nsel, pos) : nullptr;
             cp_async16(&rows_sh[buf][r * kRowStride + c * 8], src ? (const void*)(src + c * 8) : (const void*)a.raw,
                        src ? 16 : 0);
             if (c == 0) valid_sh[buf][r] = src != nullptr;
@@ -98,7 +126,7 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
         cp_async_commit();
     };
 
-    if (nblk > 0) gather(0, 0);
+    if (gb_lo < gb_hi) gather(gb_lo, 0);
 
     // Q fragments for this warp's 16 heads: 8 k-steps of 16 dims.
     uint32_t qa[8][4];
@@ -114,15 +142,26 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
         }
     }
 
+    // per-split state (fresh at every split start)
     float o[16][4];
+    float mrow[2], lrow[2];
+    // running fold over splits (FUSED only)
+    float Of[FUSED ? 16 : 1][4];
+    float Mf[2] = {-INFINITY, -INFINITY}, Lf[2] = {0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
+    for (int j = 0; j < (FUSED ? 16 : 1); ++j) Of[j][0] = Of[j][1] = Of[j][2] = Of[j][3] = 0.f;
+    auto reset_split = [&]() {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        mrow[0] = mrow[1] = -INFINITY;
+        lrow[0] = lrow[1] = 0.f;
+    };
+    reset_split();
 
-    for (int blk = 0; blk < nblk; ++blk) {
-        const int buf = blk & 1;
-        if (blk + 1 < nblk) {
-            gather(blk + 1, buf ^ 1);
+    for (int gb = gb_lo; gb < gb_hi; ++gb) {
+        const int buf = (gb - gb_lo) & 1;
+        if (gb + 1 < gb_hi) {
+            gather(gb + 1, buf ^ 1);
             cp_async_wait<1>();
         } else {
             cp_async_wait<0>();
@@ -212,31 +251,66 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a) {
             }
         }
         __syncthreads();  // buffer `buf` is refilled two blocks later
+
+        if constexpr (FUSED) {
+            if ((gb + 1) % bps == 0 || gb + 1 == gb_hi) {   // end of a split: fold, start the next
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    float Mn, fa, fb;
+                    fold_scales(Mf[h2], mrow[h2], Mn, fa, fb);
+                    Lf[h2] = fold_val(Lf[h2], fa, lrow[h2], fb);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        Of[j][2 * h2] = fold_val(Of[j][2 * h2], fa, o[j][2 * h2], fb);
+                        Of[j][2 * h2 + 1] = fold_val(Of[j][2 * h2 + 1], fa, o[j][2 * h2 + 1], fb);
+                    }
+                    Mf[h2] = Mn;
+                }
+                reset_split();
+            }
+        }
     }
 
-    // split partials
     const int h0 = warp * 16 + g;
-    float* po = a.part_o + (((int64_t)t * a.nsplit + sp) * H) * 128;
+    if constexpr (FUSED) {
+        bf16* ob = out + ((int64_t)t * H) * 128;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        const int c = 8 * j + 2 * tq;
-        *reinterpret_cast<float2*>(po + (int64_t)h0 * 128 + c) = make_float2(o[j][0], o[j][1]);
-        *reinterpret_cast<float2*>(po + (int64_t)(h0 + 8) * 128 + c) = make_float2(o[j][2], o[j][3]);
-    }
-    if (tq == 0) {
-        float* pm = a.part_ml + (((int64_t)t * a.nsplit + sp) * H) * 2;
-        pm[h0 * 2] = mrow[0];
-        pm[h0 * 2 + 1] = lrow[0];
-        pm[(h0 + 8) * 2] = mrow[1];
-        pm[(h0 + 8) * 2 + 1] = lrow[1];
+        for (int j = 0; j < 16; ++j) {
+            const int c = 8 * j + 2 * tq;
+            *reinterpret_cast<uint32_t*>(ob + (int64_t)h0 * 128 + c) =
+                pack_bf16(fin_out(Of[j][0], Lf[0]), fin_out(Of[j][1], Lf[0]));
+            *reinterpret_cast<uint32_t*>(ob + (int64_t)(h0 + 8) * 128 + c) =
+                pack_bf16(fin_out(Of[j][2], Lf[1]), fin_out(Of[j][3], Lf[1]));
+        }
+        if (lse && tq == 0) {
+            lse[(int64_t)t * H + h0] = fin_lse(Mf[0], Lf[0]);
+            lse[(int64_t)t * H + h0 + 8] = fin_lse(Mf[1], Lf[1]);
+        }
+    } else {
+        // split partial (an empty split leaves m = -inf, l = 0, o = 0)
+        const int sp = blockIdx.x;
+        float* po = a.part_o + (((int64_t)t * a.nsplit + sp) * H) * 128;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int c = 8 * j + 2 * tq;
+            *reinterpret_cast<float2*>(po + (int64_t)h0 * 128 + c) = make_float2(o[j][0], o[j][1]);
+            *reinterpret_cast<float2*>(po + (int64_t)(h0 + 8) * 128 + c) = make_float2(o[j][2], o[j][3]);
+        }
+        if (tq == 0) {
+            float* pm = a.part_ml + (((int64_t)t * a.nsplit + sp) * H) * 2;
+            pm[h0 * 2] = mrow[0];
+            pm[h0 * 2 + 1] = lrow[0];
+            pm[(h0 + 8) * 2] = mrow[1];
+            pm[(h0 + 8) * 2 + 1] = lrow[1];
+        }
     }
     griddep_trigger();
 }
 
-// Merge of the split partials of one (query, head) per warp: lane i holds
-// split i's (max, sum) -- 32 splits per pass, passes merged in order -- and
-// every lane owns 4 output channels, issuing all its splits' partial-output
-// loads before summing them in split order.  grid (H / 4, T), 128 threads.
+// Fold of the split partials of one (query, head) per warp, in split order
+// (fold_split above): lane i holds split i's (max, sum) -- 32 splits per
+// pass -- and every lane owns 4 output channels, issuing all its splits'
+// partial-output loads before folding them.  grid (H / 4, T), 128 threads.
 __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                                                       int nsplit, int H, bf16* __restrict__ out,
                                                       float* __restrict__ lse) {
@@ -244,26 +318,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
     const int h = blockIdx.x * 4 + warp, t = blockIdx.y;
     griddep_wait();
     if (h >= H) return;
-    // pass 1: the global max
-    float M = -INFINITY;
-    for (int base = 0; base < nsplit; base += 32) {
-        const int i = base + lane;
-        const float mi = i < nsplit ? part_ml[(((int64_t)t * nsplit + i) * H + h) * 2] : -INFINITY;
-        M = fmaxf(M, mi);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    // pass 2: factors, sum and output, 32 splits at a time in split order
-    float L = 0.f;
+    float M = -INFINITY, L = 0.f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int base = 0; base < nsplit; base += 32) {
         const int i = base + lane;
-        float f = 0.f, li = 0.f;
+        float mi = -INFINITY, li = 0.f;
         if (i < nsplit) {
             const int64_t o = (((int64_t)t * nsplit + i) * H + h) * 2;
-            const float mi = part_ml[o];
+            mi = part_ml[o];
             li = part_ml[o + 1];
-            f = (M == -INFINITY || mi == -INFINITY) ? 0.f : exp2f(mi - M);
         }
         const int cnt = min(32, nsplit - base);
         float4 ov[32];
@@ -275,21 +338,23 @@ __global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ 
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             if (j < cnt) {
-                const float fj = __shfl_sync(0xffffffffu, f, j);
+                const float mj = __shfl_sync(0xffffffffu, mi, j);
                 const float lj = __shfl_sync(0xffffffffu, li, j);
-                L = fmaf(lj, fj, L);
-                O.x = fmaf(ov[j].x, fj, O.x);
-                O.y = fmaf(ov[j].y, fj, O.y);
-                O.z = fmaf(ov[j].z, fj, O.z);
-                O.w = fmaf(ov[j].w, fj, O.w);
+                float Mn, fa, fb;
+                fold_scales(M, mj, Mn, fa, fb);
+                L = fold_val(L, fa, lj, fb);
+                O.x = fold_val(O.x, fa, ov[j].x, fb);
+                O.y = fold_val(O.y, fa, ov[j].y, fb);
+                O.z = fold_val(O.z, fa, ov[j].z, fb);
+                O.w = fold_val(O.w, fa, ov[j].w, fb);
+                M = Mn;
             }
         }
     }
     bf16* op = out + ((int64_t)t * H + h) * 128 + lane * 4;
-    const float r0 = L > 0.f ? O.x / L : 0.f, r1 = L > 0.f ? O.y / L : 0.f;
-    const float r2 = L > 0.f ? O.z / L : 0.f, r3 = L > 0.f ? O.w / L : 0.f;
-    *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16(r0, r1), pack_bf16(r2, r3));
-    if (lse && lane == 0) lse[(int64_t)t * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    *reinterpret_cast<uint2*>(op) =
+        make_uint2(pack_bf16(fin_out(O.x, L), fin_out(O.y, L)), pack_bf16(fin_out(O.z, L), fin_out(O.w, L)));
+    if (lse && lane == 0) lse[(int64_t)t * H + h] = fin_lse(M, L);
     griddep_trigger();
 }
 
@@ -304,7 +369,7 @@ cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int
                           int max_blocks, int W, float scale, void* out, float* lse, float* part_o,
                           float* part_ml, unsigned* status, bool use_partials, cudaStream_t stream,
                           int* launches) {
-    (void)use_partials;   // every split writes partials that combine_kernel merges
+    (void)use_partials;   // the split shape always writes partials (fused shape: none)
     AttnArgs a;
     a.q = reinterpret_cast<const bf16*>(q);
     a.q_seq = q_seq;
@@ -325,23 +390,31 @@ cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int
     a.part_o = part_o;
     a.part_ml = part_ml;
     a.status = status;
-    dim3 grid(a.nsplit, T);
+    // Many queries: one CTA per query folds its splits itself (same result).
+    const bool fused = T >= 2 * current_sm_count() || a.nsplit == 1;
+    bf16* ob = reinterpret_cast<bf16*>(out);
     cudaError_t e = cudaSuccess;
+    auto go = [&](auto kern_split, auto kern_fused, int threads) {
+        if (fused) return launch_pdl(kern_fused, dim3(T), dim3(threads), 0, stream, a, ob, lse);
+        return launch_pdl(kern_split, dim3(a.nsplit, T), dim3(threads), 0, stream, a, ob, lse);
+    };
     switch (H) {
-        case 16: e = launch_pdl(attend_kernel<1>, grid, dim3(32), 0, stream, a); break;
-        case 32: e = launch_pdl(attend_kernel<2>, grid, dim3(64), 0, stream, a); break;
-        case 48: e = launch_pdl(attend_kernel<3>, grid, dim3(96), 0, stream, a); break;
-        case 64: e = launch_pdl(attend_kernel<4>, grid, dim3(128), 0, stream, a); break;
-        case 80: e = launch_pdl(attend_kernel<5>, grid, dim3(160), 0, stream, a); break;
-        case 96: e = launch_pdl(attend_kernel<6>, grid, dim3(192), 0, stream, a); break;
-        case 112: e = launch_pdl(attend_kernel<7>, grid, dim3(224), 0, stream, a); break;
-        case 128: e = launch_pdl(attend_kernel<8>, grid, dim3(256), 0, stream, a); break;
+        case 16: e = go(attend_kernel<1, false>, attend_kernel<1, true>, 32); break;
+        case 32: e = go(attend_kernel<2, false>, attend_kernel<2, true>, 64); break;
+        case 48: e = go(attend_kernel<3, false>, attend_kernel<3, true>, 96); break;
+        case 64: e = go(attend_kernel<4, false>, attend_kernel<4, true>, 128); break;
+        case 80: e = go(attend_kernel<5, false>, attend_kernel<5, true>, 160); break;
+        case 96: e = go(attend_kernel<6, false>, attend_kernel<6, true>, 192); break;
+        case 112: e = go(attend_kernel<7, false>, attend_kernel<7, true>, 224); break;
+        case 128: e = go(attend_kernel<8, false>, attend_kernel<8, true>, 256); break;
         default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
+    *launches += 1;
+    if (fused) return e;
     e = launch_pdl(combine_kernel, dim3((H + 3) / 4, T), dim3(128), 0, stream, (const float*)part_o,
-                   (const float*)part_ml, a.nsplit, H, reinterpret_cast<bf16*>(out), lse);
-    *launches += 2;
+                   (const float*)part_ml, a.nsplit, H, ob, lse);
+    *launches += 1;
     return e;
 }
 

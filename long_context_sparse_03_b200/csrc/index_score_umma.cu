@@ -1,0 +1,506 @@
+// index_score_umma.cu -- lightning-indexer scoring for many queries on the
+// 5th-generation tensor cores (tcgen05 / TMEM), used for chunked prefill.
+//
+// DeepSeek-V4 summary (b-lab.team), "Core Methodological Innovations" 1,
+// CSA bullet: S_j = sum_h w_h max(0, q_h . k_j) over the compressed blocks a
+// query can see.  With thousands of queries per call the scores are a dense
+// contraction: for one sequence, D[j][(t, h)] = k_j . q_{t,h} is a GEMM of
+// the key cache (M = keys) with the stacked query heads (N = queries x Hi,
+// K = 64 channels), followed by a per-query epilogue (ReLU, weighted head sum).
+//
+// One CTA owns QG = 256 / Hi consecutive queries (N = 256 columns) for the
+// whole key range, so its epilogue sees every score of those queries:
+//   * warp 8 (one lane) streams 128-key tiles of the cache into a 4-stage
+//     ring with 3-D TMA tensor copies (128-byte swizzle, the canonical K-major
+//     operand layout of the tensor core);
+//   * warp 9 (one lane) issues tcgen05.mma (M = 128 keys, N = 256, K = 16,
+//     bf16 x bf16 -> fp32) into one of two TMEM accumulators (2 x 256
+//     columns): q is split into bf16 hi + lo halves (two MMAs per k-step) so
+//     the product keeps ~16 significant bits of the fp32 query;
+//   * warps 0-7 drain an accumulator with tcgen05.ld (warp w: TMEM lanes
+//     32(w%4).., columns 128(w/4)..), release it, and form the scores:
+//     thread = key, so the head sum is in-thread; each score of a visible
+//     block is stored, and the maximum of every 32-key group goes to the
+//     query's 2048-bin histogram (the same bins as the decode kernel).
+// At the end the CTA turns its queries' histograms into threshold keys; the
+// collect and rank passes of the decode path then select the exact top-k.
+//
+// Queries of a CTA that belong to different sequences are handled in one
+// pass per distinct sequence (columns of the other sequences are ignored).
+// Every mbarrier wait is bounded: one that runs out flags CSA_DEV_TIMEOUT
+// and the CTA carries on, so it always frees its TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstddef>
+#include <mutex>
+
+#include "common.cuh"
+#include "csa.h"
+
+namespace csa {
+
+constexpr int kUmTile = 128;                      // keys per tile (MMA M)
+constexpr int kUmStages = 4;
+constexpr int kUmEpiWarps = 8;
+constexpr int kUmThreads = (kUmEpiWarps + 2) * 32;
+constexpr int kUmTileBytes = kUmTile * 128;       // 16 KB of bf16 key rows
+constexpr int kUmQBytes = 256 * 128;              // one 256 x 64 bf16 operand
+constexpr int kUmCols = 512;                      // two 256-column accumulators
+constexpr int kUmHistBins = 2048, kUmHistShift = 21;
+constexpr unsigned kUmWaitTries = 1u << 22;
+
+struct UmmaScoreArgs {
+    const float* q;       // [T][Hi][64]
+    const float* w;       // [T][Hi]
+    const int* q_seq;
+    const int* q_pos;
+    int T, m, max_blocks, k;
+    float* scores;        // [T][ld_scores]
+    int64_t ld_scores;
+    unsigned* hist;       // [T][2048]
+    unsigned* thr;        // [T]
+    unsigned* status;
+};
+
+struct UmmaSmem {
+    alignas(16) float w_sh[256];   // read as float4
+    uint64_t full[kUmStages], empty[kUmStages], acc_full[2], acc_empty[2], mma_done;
+    uint32_t tmem_base;
+    int nseq, ntiles_total;
+    int seqs[64], ntiles[64];
+    int V_sh[64], seq_sh[64];
+};
+static_assert(offsetof(UmmaSmem, w_sh) == 0, "w_sh leads the struct (16-byte aligned)");
+static_assert(offsetof(UmmaSmem, full) % 8 == 0, "mbarriers are 8-byte aligned");
+
+constexpr size_t umma_smem_bytes() { return 1024 + 2 * kUmQBytes + kUmStages * kUmTileBytes + sizeof(UmmaSmem); }
+
+// ---------------------------------------------------------------- tcgen05 / TMA wrappers
+// Shared-memory operand descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (rows of 64 bf16), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;              // leading byte offset (unused with this swizzle)
+    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset
+    d |= (uint64_t)1 << 46;              // version
+    d |= (uint64_t)2 << 61;              // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major,
+// N = 256, M = 128.
+constexpr uint32_t kUmIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kUmIdesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+// 32 consecutive TMEM columns of this warp's 32 lanes, one lane per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32], int o) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr + (uint32_t)o));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
+// 3-D tiled TMA load (x = channel, y = key row, z = sequence) into a stage.
+__device__ __forceinline__ void tma_load_keys(void* dst, const CUtensorMap* map, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];\n" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Highest bin b with (#counts in bins >= b) >= k over one query's 2048-bin
+// histogram (0 when fewer than k), by one warp: lane l sums the 64 bins
+// [2048 - 64(l+1), 2048 - 64l) and the lane where the running count from the
+// top reaches k walks its bins.
+__device__ unsigned warp_threshold_bin(const unsigned* gh, int k) {
+    const int lane = threadIdx.x & 31;
+    const unsigned* mine = gh + kUmHistBins - 64 * (lane + 1);
+    unsigned c[64];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(mine) + i);
+        c[4 * i] = v.x;
+        c[4 * i + 1] = v.y;
+        c[4 * i + 2] = v.z;
+        c[4 * i + 3] = v.w;
+    }
+    unsigned s = 0;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) s += c[i];
+    unsigned incl = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    const unsigned excl = incl - s;
+    const unsigned hit = __ballot_sync(0xffffffffu, excl < (unsigned)k && (unsigned)k <= incl);
+    unsigned b = 0;
+    if (hit) {
+        const int src = __ffs(hit) - 1;
+        unsigned bin = 0;
+        if (lane == src) {
+            unsigned run = excl;
+            for (int i = 63; i >= 0; --i) {   // from the lane's top bin down
+                run += c[i];
+                if (run >= (unsigned)k) {
+                    bin = (unsigned)(kUmHistBins - 64 * (lane + 1) + i);
+                    break;
+                }
+            }
+        }
+        b = __shfl_sync(0xffffffffu, bin, src);
+    }
+    return b;
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kUmThreads, 1)
+    index_score_umma_kernel(const __grid_constant__ CUtensorMap kmap, UmmaScoreArgs a) {
+    constexpr int QG = 256 / HI;            // queries per CTA
+    constexpr int QW = 128 / HI;            // queries per epilogue warp
+    extern __shared__ uint8_t smem_um_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_um_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* qhi = base;
+    uint8_t* qlo = base + kUmQBytes;
+    uint8_t* kst = base + 2 * kUmQBytes;
+    UmmaSmem& sm = *reinterpret_cast<UmmaSmem*>(kst + kUmStages * kUmTileBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = blockIdx.x * QG;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kUmStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], kUmEpiWarps);
+        }
+        mbar_init(&sm.mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(&sm.tmem_base)),
+                     "r"(kUmCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    griddep_wait();
+
+    // q as bf16 hi + lo operands (row n = query * HI + head, 128-byte
+    // swizzle: 16-byte chunk c of row n sits at chunk c ^ (n % 8)), w, and
+    // the queries' visibility and sequence.
+    for (int i = threadIdx.x; i < 256 * 8; i += kUmThreads) {
+        const int n = i >> 3, c = i & 7, ql = n / HI, h = n % HI, t = t0 + ql;
+        float x[8];
+        if (t < a.T) {
+            const float4* src = reinterpret_cast<const float4*>(a.q + ((int64_t)t * HI + h) * 64 + c * 8);
+            const float4 u0 = src[0], u1 = src[1];
+            x[0] = u0.x; x[1] = u0.y; x[2] = u0.z; x[3] = u0.w;
+            x[4] = u1.x; x[5] = u1.y; x[6] = u1.z; x[7] = u1.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.f;
+        }
+        uint4 vh, vl;
+        uint32_t* ph = reinterpret_cast<uint32_t*>(&vh);
+        uint32_t* pl = reinterpret_cast<uint32_t*>(&vl);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float h0 = __bfloat162float(__float2bfloat16_rn(x[2 * e]));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(x[2 * e + 1]));
+            ph[e] = pack_bf16(h0, h1);
+            pl[e] = pack_bf16(x[2 * e] - h0, x[2 * e + 1] - h1);
+        }
+        const int off = n * 128 + ((c ^ (n & 7)) << 4);
+        *reinterpret_cast<uint4*>(qhi + off) = vh;
+        *reinterpret_cast<uint4*>(qlo + off) = vl;
+    }
+    for (int i = threadIdx.x; i < 256; i += kUmThreads) {
+        const int t = t0 + i / HI;
+        sm.w_sh[i] = t < a.T ? a.w[(int64_t)t * HI + i % HI] : 0.f;
+    }
+    if (threadIdx.x < QG) {
+        const int t = t0 + threadIdx.x;
+        const bool ok = t < a.T;
+        sm.V_sh[threadIdx.x] = ok ? min((a.q_pos[t] + 1) / a.m, a.max_blocks) : 0;
+        sm.seq_sh[threadIdx.x] = ok ? a.q_seq[t] : -1;
+    }
+    fence_proxy_async();   // generic-proxy writes of the q operands -> tensor core
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+        // one pass per distinct sequence, in order of first appearance
+        int ns = 0, tot = 0;
+        for (int i = 0; i < QG; ++i) {
+            const int s = sm.seq_sh[i];
+            if (s < 0) continue;
+            bool seen = false;
+            for (int j = 0; j < ns; ++j) seen |= sm.seqs[j] == s;
+            if (seen) continue;
+            int vmax = 0;
+            for (int j = i; j < QG; ++j)
+                if (sm.seq_sh[j] == s) vmax = max(vmax, sm.V_sh[j]);
+            sm.seqs[ns] = s;
+            sm.ntiles[ns] = (vmax + kUmTile - 1) / kUmTile;
+            tot += sm.ntiles[ns];
+            ++ns;
+        }
+        sm.nseq = ns;
+        sm.ntiles_total = tot;
+    }
+    __syncthreads();
+    const uint32_t tmem = sm.tmem_base;
+    const int nseq = sm.nseq, ntot = sm.ntiles_total;
+
+    if (warp == kUmEpiWarps) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int slot = 0;
+            unsigned ph = 0;
+            int it = 0;
+            for (int p = 0; p < nseq; ++p) {
+                for (int j = 0; j < sm.ntiles[p]; ++j, ++it) {
+                    if (it >= kUmStages && !mbar_wait_bounded(&sm.empty[slot], ph ^ 1u, kUmWaitTries))
+                        flag_status(a.status, kDevTimeout);
+                    mbar_arrive_expect_tx(&sm.full[slot], kUmTileBytes);
+                    tma_load_keys(kst + slot * kUmTileBytes, &kmap, j * kUmTile, sm.seqs[p], &sm.full[slot]);
+                    if (++slot == kUmStages) {
+                        slot = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            // drain: the last load of every stage has landed
+            for (int s = 0; s < kUmStages && s < ntot; ++s) {
+                const int last = s + ((ntot - 1 - s) / kUmStages) * kUmStages;
+                if (!mbar_wait_bounded(&sm.full[s], (unsigned)(last / kUmStages) & 1u, kUmWaitTries))
+                    flag_status(a.status, kDevTimeout);
+            }
+        }
+    } else if (warp == kUmEpiWarps + 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int slot = 0, abuf = 0;
+            unsigned ph = 0, aph = 0;
+            const uint32_t qh = smem_u32(qhi), qlw = smem_u32(qlo);
+            for (int it = 0; it < ntot; ++it) {
+                bool ok = mbar_wait_bounded(&sm.full[slot], ph, kUmWaitTries);
+                if (it >= 2) ok &= mbar_wait_bounded(&sm.acc_empty[abuf], aph ^ 1u, kUmWaitTries);
+                if (!ok) flag_status(a.status, kDevTimeout);
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(abuf * 256);
+                const uint32_t ka = smem_u32(kst + slot * kUmTileBytes);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) umma_bf16(d, sw128_desc(ka + 32 * s), sw128_desc(qh + 32 * s), s > 0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) umma_bf16(d, sw128_desc(ka + 32 * s), sw128_desc(qlw + 32 * s), 1);
+                umma_commit(&sm.empty[slot]);
+                umma_commit(&sm.acc_full[abuf]);
+                if (++slot == kUmStages) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
+                if (++abuf == 2) {
+                    abuf = 0;
+                    aph ^= 1u;
+                }
+            }
+            umma_commit(&sm.mma_done);
+        }
+    } else {
+        // ------------------------------------------------ epilogue warps
+        const int quarter = warp & 3, half = warp >> 2;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        constexpr int LOGQ = QW == 32 ? 5 : QW == 16 ? 4 : 3;
+        const int my_q = lane >> (5 - LOGQ);                        // query slot this lane reduces
+        const bool my_red = (lane & ((1 << (5 - LOGQ)) - 1)) == 0;  // one lane per slot writes
+        int abuf = 0;
+        unsigned aph = 0;
+        for (int p = 0; p < nseq; ++p) {
+            const int seq = sm.seqs[p];
+            int vq[QW];   // visible blocks of each query of this warp in this pass (0: other sequence)
+#pragma unroll
+            for (int qi = 0; qi < QW; ++qi) {
+                const int ql = half * QW + qi;
+                vq[qi] = sm.seq_sh[ql] == seq ? sm.V_sh[ql] : 0;
+            }
+            const int t_red = t0 + half * QW + my_q;
+            const int v_red = sm.seq_sh[half * QW + my_q] == seq ? sm.V_sh[half * QW + my_q] : 0;
+            for (int j = 0; j < sm.ntiles[p]; ++j) {
+                const bool ok = mbar_wait_bounded(&sm.acc_full[abuf], aph, kUmWaitTries);
+                if (!ok && lane == 0) flag_status(a.status, kDevTimeout);
+                tc_fence_after();
+                uint32_t r[4][32];
+                const uint32_t col = tmem + lane_base + (uint32_t)(abuf * 256 + half * 128);
+                tmem_ld32(col, r[0], 0);
+                tmem_ld32(col, r[1], 32);
+                tmem_ld32(col, r[2], 64);
+                tmem_ld32(col, r[3], 96);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
+                if (++abuf == 2) {
+                    abuf = 0;
+                    aph ^= 1u;
+                }
+                if (!ok) continue;
+                const int g0 = j * kUmTile + quarter * 32;   // first key of this warp's 32-key group
+                const int key = g0 + lane;
+                // scores of the lane's key for the warp's queries (masked, no branches)
+                float sc[QW];
+#pragma unroll
+                for (int qi = 0; qi < QW; ++qi) {
+                    const float4* wp = reinterpret_cast<const float4*>(&sm.w_sh[(half * QW + qi) * HI]);
+                    float s = 0.f;
+#pragma unroll
+                    for (int h4 = 0; h4 < HI / 4; ++h4) {
+                        const float4 wv = wp[h4];
+                        const int c = qi * HI + h4 * 4;
+                        s = fmaf(wv.x, fmaxf(__uint_as_float(r[c >> 5][c & 31]), 0.f), s);
+                        s = fmaf(wv.y, fmaxf(__uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]), 0.f), s);
+                        s = fmaf(wv.z, fmaxf(__uint_as_float(r[(c + 2) >> 5][(c + 2) & 31]), 0.f), s);
+                        s = fmaf(wv.w, fmaxf(__uint_as_float(r[(c + 3) >> 5][(c + 3) & 31]), 0.f), s);
+                    }
+                    sc[qi] = s;
+                    if (key < vq[qi]) a.scores[(int64_t)(t0 + half * QW + qi) * a.ld_scores + key] = s;
+                }
+                if (a.hist) {
+                    // maximum over the 32 keys of every query: halving exchange, after
+                    // which lane l holds query slot l >> (5 - LOGQ)
+#pragma unroll
+                    for (int qi = 0; qi < QW; ++qi)
+                        if (!(key < vq[qi])) sc[qi] = -INFINITY;
+                    int n = QW;
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) {
+                        if (n > 1) {
+                            const bool upper = (lane & o) != 0;
+#pragma unroll
+                            for (int i = 0; i < QW / 2; ++i) {
+                                if (i < n / 2) {
+                                    const float send = upper ? sc[i] : sc[i + n / 2];
+                                    const float keep = upper ? sc[i + n / 2] : sc[i];
+                                    sc[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                                }
+                            }
+                            n >>= 1;
+                        } else {
+                            sc[0] = fmaxf(sc[0], __shfl_xor_sync(0xffffffffu, sc[0], o));
+                        }
+                    }
+                    if (my_red && g0 < v_red)
+                        atomicAdd(&a.hist[(int64_t)t_red * kUmHistBins + (score_key(sc[0]) >> kUmHistShift)], 1u);
+                }
+            }
+        }
+        // every histogram count of this CTA's queries is in: threshold keys
+        __threadfence();
+        named_sync(1, kUmEpiWarps * 32);
+        for (int ql = warp; ql < QG && a.hist; ql += kUmEpiWarps) {
+            const int t = t0 + ql;
+            if (t >= a.T) break;
+            const unsigned b = warp_threshold_bin(a.hist + (int64_t)t * kUmHistBins, a.k);
+            if (lane == 0) a.thr[t] = b << kUmHistShift;
+        }
+    }
+
+    // teardown: every MMA has completed before TMEM is freed
+    __syncthreads();
+    if (warp == 0) {
+        if (ntot > 0 && !mbar_wait_bounded(&sm.mma_done, 0, kUmWaitTries)) {
+            if (lane == 0) flag_status(a.status, kDevTimeout);
+        }
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kUmCols) : "memory");
+    }
+    griddep_trigger();
+}
+
+// ---------------------------------------------------------------- host
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Whether the tensor-core path takes this call (else the decode kernel does).
+bool index_score_umma_applies(int T, int Hi, int fmt, const float* q, const void* kidx, int64_t kstride_bytes) {
+    return fmt == 0 && (Hi == 4 || Hi == 8 || Hi == 16) && T >= 256 && (reinterpret_cast<uintptr_t>(kidx) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(q) & 15) == 0 &&
+           kstride_bytes % 16 == 0 && kstride_bytes > 0 && tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_index_score_umma(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
+                                    const void* kidx, int64_t kstride_bytes, int m, int max_blocks, int k,
+                                    float* scores, int64_t ld_scores, unsigned* hist, unsigned* thr, unsigned* status,
+                                    cudaStream_t stream) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map;
+    // key cache as a 3-D tensor: 64 channels x max_blocks rows x sequences
+    // (rows past max_blocks read as zeros; the sequence extent is only a bound)
+    const cuuint64_t dims[3] = {64, (cuuint64_t)max_blocks, (cuuint64_t)CSA_MAX_T};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)kstride_bytes};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kUmTile, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kidx), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    UmmaScoreArgs a;
+    a.q = q;
+    a.w = w;
+    a.q_seq = q_seq;
+    a.q_pos = q_pos;
+    a.T = T;
+    a.m = m;
+    a.max_blocks = max_blocks;
+    a.k = k;
+    a.scores = scores;
+    a.ld_scores = ld_scores;
+    a.hist = hist;
+    a.thr = thr;
+    a.status = status;
+    const size_t smem = umma_smem_bytes();
+    auto go = [&](auto kern, int qg) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, dim3((unsigned)((T + qg - 1) / qg)), dim3(kUmThreads), smem, stream, map, a);
+    };
+    if (Hi == 4) return go(index_score_umma_kernel<4>, 64);
+    if (Hi == 8) return go(index_score_umma_kernel<8>, 32);
+    return go(index_score_umma_kernel<16>, 16);
+}
+
+}  // namespace csa

@@ -158,8 +158,10 @@ def _keys_f64(oracle, keys, kscale, fmt):
     return oracle.e4m3_decode(keys) * kscale[..., None].astype(np.float64)
 
 
+# T >= 256 with bf16 keys and Hi in {4, 8, 16} runs the tensor-core (tcgen05)
+# scoring kernel; the queries of those cases mix two sequences.
 @pytest.mark.parametrize("fmt,Hi,N,T", [(0, 8, 5000, 6), (1, 8, 5000, 6), (0, 4, 1024, 1), (0, 16, 3000, 4),
-                                        (1, 3, 2100, 3)])
+                                        (1, 3, 2100, 3), (0, 8, 3000, 300), (0, 4, 2000, 260), (0, 16, 1500, 256)])
 def test_index_scores(oracle, fmt, Hi, N, T):
     rng = np.random.default_rng(fmt * 10 + Hi + N)
     m = 4
@@ -180,7 +182,8 @@ def test_index_scores(oracle, fmt, Hi, N, T):
 @pytest.mark.parametrize("fmt,Hi,N,T,k,ties,neg", [
     (0, 8, 5000, 6, 64, False, False), (0, 8, 9000, 3, 512, False, False), (1, 8, 9000, 3, 512, False, False),
     (0, 4, 1024, 1, 64, False, False), (0, 8, 3000, 4, 2048, False, False), (0, 8, 2500, 5, 1, False, False),
-    (0, 8, 4000, 4, 100, True, False), (0, 8, 4000, 4, 300, False, True), (1, 16, 20000, 2, 1024, False, False)])
+    (0, 8, 4000, 4, 100, True, False), (0, 8, 4000, 4, 300, False, True), (1, 16, 20000, 2, 1024, False, False),
+    (0, 8, 3000, 300, 256, False, False), (0, 8, 4000, 260, 100, True, False), (0, 16, 2500, 300, 512, False, True)])
 def test_index_select(oracle, fmt, Hi, N, T, k, ties, neg):
     rng = np.random.default_rng(1000 + fmt + Hi + N + k)
     m = 4
@@ -199,6 +202,31 @@ def test_index_select(oracle, fmt, Hi, N, T, k, ties, neg):
     for t in range(T):
         V = min((q_pos[t] + 1) // m, N)
         A = score_scale(q[t].astype(np.float64), w[t].astype(np.float64), kf[q_seq[t]])
+        check_topk(gi[t], gs[t], S[t], A, V, k)
+
+
+def test_index_select_prefill_chunk(oracle):
+    """A causal chunk of one sequence (consecutive positions, the prefill
+    layout) on the tensor-core scoring path: every query judged."""
+    rng = np.random.default_rng(77)
+    m, Hi, N, k, T = 4, 8, 2600, 300, 640
+    keys, _, q, w, _, _ = _index_case(oracle, rng, 1, N, Hi, 1, 0)
+    q = rng.standard_normal((T, Hi, 64)).astype(np.float32)
+    w = rng.standard_normal((T, Hi)).astype(np.float32)
+    q_seq = np.zeros(T, np.int32)
+    q_pos = (N * m - T + np.arange(T)).astype(np.int32)
+    S = oracle.index_scores(q.astype(np.float64), w.astype(np.float64), q_seq, q_pos, keys, m, N)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_index_workspace_size(T, 0, Hi, k, N))
+    csa.csa_index_select(torch.from_numpy(q).cuda(), torch.from_numpy(w).cuda(), dev_i32(q_seq), dev_i32(q_pos),
+                         dev_bf16(keys), m, N, k, idx, sc, ws)
+    ws.check()
+    gi, gs = idx.cpu().numpy(), sc.cpu().numpy()
+    kf = bf16_bits_to_f64(keys)
+    for t in range(T):
+        V = min((q_pos[t] + 1) // m, N)
+        A = score_scale(q[t].astype(np.float64), w[t].astype(np.float64), kf[0])
         check_topk(gi[t], gs[t], S[t], A, V, k)
 
 
@@ -350,6 +378,49 @@ def test_batch_invariance_and_determinism(oracle):
         alone = run(np.array([t]))
         for a, b in zip(full, alone):
             assert np.array_equal(a[t], b[0], equal_nan=True)
+
+
+@pytest.mark.parametrize("dense", [False, True], ids=["csa", "hca"])
+def test_attend_launch_shapes_bit_identical(oracle, dense):
+    """Many queries run one CTA per query that folds its splits itself; a few
+    queries run one CTA per split plus the combine pass.  Both fold the same
+    per-split partials in the same order, so a query's output and lse are
+    bitwise the same in either shape; sampled queries also meet the oracle."""
+    rng = np.random.default_rng(404 + dense)
+    m, H, W, T = (16, 64, 128, 400) if dense else (4, 64, 128, 400)
+    B, N = 3, 700
+    k = 0 if dense else 300
+    q, comp, raw, q_seq, q_pos, idx = _attn_case(rng, B, N, N * m, H, T, max(k, 1), W, m)
+    cd, rd = dev_bf16(comp), dev_bf16(raw)
+
+    def run(sel):
+        Tn = len(sel)
+        out = torch.empty((Tn, H, 128), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((Tn, H), dtype=torch.float32, device="cuda")
+        if dense:
+            wa = csa.Workspace(csa.hca_attend_workspace_size(Tn, H, N + W))
+            csa.hca_attend(dev_bf16(q[sel]), dev_i32(q_seq[sel]), dev_i32(q_pos[sel]), cd, rd, m, N, W, 128 ** -0.5,
+                           out, lse, wa)
+        else:
+            wa = csa.Workspace(csa.csa_attend_workspace_size(Tn, H, k + W))
+            csa.csa_sparse_attend(dev_bf16(q[sel]), dev_i32(q_seq[sel]), dev_i32(q_pos[sel]), cd, rd, m,
+                                  torch.from_numpy(np.ascontiguousarray(idx[sel, :k])).cuda(), W, 128 ** -0.5, out,
+                                  lse, wa)
+        wa.check()
+        return host_bits(out), lse.cpu().numpy()
+
+    full_o, full_l = run(np.arange(T))
+    picks = np.array([0, 1, 2, 177, T - 1])
+    few_o, few_l = run(picks)
+    assert np.array_equal(full_o[picks], few_o)
+    assert np.array_equal(full_l[picks], few_l, equal_nan=True)
+    for t in (0, 177):
+        if dense:
+            ro, rl = oracle.hca_attend(q[t:t + 1], q_seq[t:t + 1], q_pos[t:t + 1], comp, raw, m, W, 128 ** -0.5)
+        else:
+            ro, rl = oracle.sparse_attend(q[t:t + 1], q_seq[t:t + 1], q_pos[t:t + 1], comp, raw, m,
+                                          np.ascontiguousarray(idx[t:t + 1, :k]), W, 128 ** -0.5)
+        check_attention(bf16_bits_to_f64(full_o[t:t + 1]), full_l[t:t + 1].astype(np.float64), ro, rl)
 
 
 @pytest.mark.parametrize("fmt", [0, 1])
