@@ -95,11 +95,25 @@ __device__ __forceinline__ float fin_lse(float M, float L) {
 // registers, output written directly.  The row blocks of consecutive splits
 // form one sequence, so the gather of the next block (cp.async, double
 // buffered) overlaps the current one across split boundaries too.
+// Dynamic shared memory: two row buffers, their valid flags and, for the
+// fused shape, the running fold of every thread (16 float4 per thread).
+constexpr int kRowsBytes = 2 * kRowBlock * kRowStride * 2;
+constexpr int kValidBytes = 2 * kRowBlock * 4;
 template <int NW, bool FUSED>
-__global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a, bf16* __restrict__ out, float* __restrict__ lse) {
+constexpr size_t attend_smem_bytes() {
+    return (size_t)kRowsBytes + kValidBytes + (FUSED ? (size_t)NW * 16 * 32 * 16 : 0);
+}
+
+template <int NW, bool FUSED>
+__global__ void __launch_bounds__(NW * 32, NW <= 4 ? 3 : 1)
+    attend_kernel(AttnArgs a, bf16* __restrict__ out, float* __restrict__ lse) {
     constexpr int H = NW * 16;
-    __shared__ __align__(16) bf16 rows_sh[2][kRowBlock * kRowStride];
-    __shared__ int valid_sh[2][kRowBlock];
+    extern __shared__ __align__(16) uint8_t att_smem[];
+    bf16 (*rows_sh)[kRowBlock * kRowStride] = reinterpret_cast<bf16 (*)[kRowBlock * kRowStride]>(att_smem);
+    int (*valid_sh)[kRowBlock] = reinterpret_cast<int (*)[kRowBlock]>(att_smem + kRowsBytes);
+    // fold slot [warp][j][lane]: this thread's 4 outputs of n-tile j
+    float4* fold_sh = reinterpret_cast<float4*>(att_smem + kRowsBytes + kValidBytes) +
+                      (threadIdx.x >> 5) * 16 * 32 + (threadIdx.x & 31);
 
     const int t = FUSED ? blockIdx.x : blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
@@ -145,11 +159,12 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a, bf16* __res
     // per-split state (fresh at every split start)
     float o[16][4];
     float mrow[2], lrow[2];
-    // running fold over splits (FUSED only)
-    float Of[FUSED ? 16 : 1][4];
+    // running fold over splits (FUSED only): outputs in fold_sh, max / sum here
     float Mf[2] = {-INFINITY, -INFINITY}, Lf[2] = {0.f, 0.f};
+    if constexpr (FUSED) {
 #pragma unroll
-    for (int j = 0; j < (FUSED ? 16 : 1); ++j) Of[j][0] = Of[j][1] = Of[j][2] = Of[j][3] = 0.f;
+        for (int j = 0; j < 16; ++j) fold_sh[j * 32] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     auto reset_split = [&]() {
 #pragma unroll
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -254,17 +269,22 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a, bf16* __res
 
         if constexpr (FUSED) {
             if ((gb + 1) % bps == 0 || gb + 1 == gb_hi) {   // end of a split: fold, start the next
+                float fa[2], fb[2];
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
-                    float Mn, fa, fb;
-                    fold_scales(Mf[h2], mrow[h2], Mn, fa, fb);
-                    Lf[h2] = fold_val(Lf[h2], fa, lrow[h2], fb);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        Of[j][2 * h2] = fold_val(Of[j][2 * h2], fa, o[j][2 * h2], fb);
-                        Of[j][2 * h2 + 1] = fold_val(Of[j][2 * h2 + 1], fa, o[j][2 * h2 + 1], fb);
-                    }
+                    float Mn;
+                    fold_scales(Mf[h2], mrow[h2], Mn, fa[h2], fb[h2]);
+                    Lf[h2] = fold_val(Lf[h2], fa[h2], lrow[h2], fb[h2]);
                     Mf[h2] = Mn;
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float4 v = fold_sh[j * 32];
+                    v.x = fold_val(v.x, fa[0], o[j][0], fb[0]);
+                    v.y = fold_val(v.y, fa[0], o[j][1], fb[0]);
+                    v.z = fold_val(v.z, fa[1], o[j][2], fb[1]);
+                    v.w = fold_val(v.w, fa[1], o[j][3], fb[1]);
+                    fold_sh[j * 32] = v;
                 }
                 reset_split();
             }
@@ -277,10 +297,10 @@ __global__ void __launch_bounds__(NW * 32) attend_kernel(AttnArgs a, bf16* __res
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int c = 8 * j + 2 * tq;
-            *reinterpret_cast<uint32_t*>(ob + (int64_t)h0 * 128 + c) =
-                pack_bf16(fin_out(Of[j][0], Lf[0]), fin_out(Of[j][1], Lf[0]));
+            const float4 v = fold_sh[j * 32];
+            *reinterpret_cast<uint32_t*>(ob + (int64_t)h0 * 128 + c) = pack_bf16(fin_out(v.x, Lf[0]), fin_out(v.y, Lf[0]));
             *reinterpret_cast<uint32_t*>(ob + (int64_t)(h0 + 8) * 128 + c) =
-                pack_bf16(fin_out(Of[j][2], Lf[1]), fin_out(Of[j][3], Lf[1]));
+                pack_bf16(fin_out(v.z, Lf[1]), fin_out(v.w, Lf[1]));
         }
         if (lse && tq == 0) {
             lse[(int64_t)t * H + h0] = fin_lse(Mf[0], Lf[0]);
@@ -394,21 +414,31 @@ cudaError_t launch_attend(const void* q, const int* q_seq, const int* q_pos, int
     const bool fused = T >= 2 * current_sm_count() || a.nsplit == 1;
     bf16* ob = reinterpret_cast<bf16*>(out);
     cudaError_t e = cudaSuccess;
-    auto go = [&](auto kern_split, auto kern_fused, int threads) {
-        if (fused) return launch_pdl(kern_fused, dim3(T), dim3(threads), 0, stream, a, ob, lse);
-        return launch_pdl(kern_split, dim3(a.nsplit, T), dim3(threads), 0, stream, a, ob, lse);
+    auto go = [&](auto kern_split, auto kern_fused, int threads, size_t smem_split, size_t smem_fused) {
+        auto kern = fused ? kern_fused : kern_split;
+        const size_t smem = fused ? smem_fused : smem_split;
+        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e2 != cudaSuccess) return e2;
+        if (fused) return launch_pdl(kern, dim3(T), dim3(threads), smem, stream, a, ob, lse);
+        return launch_pdl(kern, dim3(a.nsplit, T), dim3(threads), smem, stream, a, ob, lse);
     };
+#define CSA_ATTEND_CASE(NWV) \
+    case NWV * 16: \
+        e = go(attend_kernel<NWV, false>, attend_kernel<NWV, true>, NWV * 32, attend_smem_bytes<NWV, false>(), \
+               attend_smem_bytes<NWV, true>()); \
+        break;
     switch (H) {
-        case 16: e = go(attend_kernel<1, false>, attend_kernel<1, true>, 32); break;
-        case 32: e = go(attend_kernel<2, false>, attend_kernel<2, true>, 64); break;
-        case 48: e = go(attend_kernel<3, false>, attend_kernel<3, true>, 96); break;
-        case 64: e = go(attend_kernel<4, false>, attend_kernel<4, true>, 128); break;
-        case 80: e = go(attend_kernel<5, false>, attend_kernel<5, true>, 160); break;
-        case 96: e = go(attend_kernel<6, false>, attend_kernel<6, true>, 192); break;
-        case 112: e = go(attend_kernel<7, false>, attend_kernel<7, true>, 224); break;
-        case 128: e = go(attend_kernel<8, false>, attend_kernel<8, true>, 256); break;
+        CSA_ATTEND_CASE(1)
+        CSA_ATTEND_CASE(2)
+        CSA_ATTEND_CASE(3)
+        CSA_ATTEND_CASE(4)
+        CSA_ATTEND_CASE(5)
+        CSA_ATTEND_CASE(6)
+        CSA_ATTEND_CASE(7)
+        CSA_ATTEND_CASE(8)
         default: return cudaErrorInvalidValue;
     }
+#undef CSA_ATTEND_CASE
     if (e != cudaSuccess) return e;
     *launches += 1;
     if (fused) return e;

@@ -10,15 +10,15 @@
 //
 // One CTA owns QG = 256 / Hi consecutive queries (N = 256 columns) for the
 // whole key range, so its epilogue sees every score of those queries:
-//   * warp 8 (one lane) streams 128-key tiles of the cache into a 4-stage
+//   * warp 16 (one lane) streams 128-key tiles of the cache into a 4-stage
 //     ring with 3-D TMA tensor copies (128-byte swizzle, the canonical K-major
 //     operand layout of the tensor core);
-//   * warp 9 (one lane) issues tcgen05.mma (M = 128 keys, N = 256, K = 16,
+//   * warp 17 (one lane) issues tcgen05.mma (M = 128 keys, N = 256, K = 16,
 //     bf16 x bf16 -> fp32) into one of two TMEM accumulators (2 x 256
 //     columns): q is split into bf16 hi + lo halves (two MMAs per k-step) so
 //     the product keeps ~16 significant bits of the fp32 query;
-//   * warps 0-7 drain an accumulator with tcgen05.ld (warp w: TMEM lanes
-//     32(w%4).., columns 128(w/4)..), release it, and form the scores:
+//   * warps 0-15 drain an accumulator with tcgen05.ld (warp w: TMEM lanes
+//     32(w%4).., columns 64(w/4)..), release it, and form the scores:
 //     thread = key, so the head sum is in-thread; each score of a visible
 //     block is stored, and the maximum of every 32-key group goes to the
 //     query's 2048-bin histogram (the same bins as the decode kernel).
@@ -42,7 +42,7 @@ namespace csa {
 
 constexpr int kUmTile = 128;                      // keys per tile (MMA M)
 constexpr int kUmStages = 4;
-constexpr int kUmEpiWarps = 8;
+constexpr int kUmEpiWarps = 16;                  // 4 per SM sub-partition
 constexpr int kUmThreads = (kUmEpiWarps + 2) * 32;
 constexpr int kUmTileBytes = kUmTile * 128;       // 16 KB of bf16 key rows
 constexpr int kUmQBytes = 256 * 128;              // one 256 x 64 bf16 operand
@@ -70,6 +70,7 @@ struct UmmaSmem {
     int nseq, ntiles_total;
     int seqs[64], ntiles[64];
     int V_sh[64], seq_sh[64];
+    int Vp[64];   // visible blocks per query in the current pass (0: another sequence)
 };
 static_assert(offsetof(UmmaSmem, w_sh) == 0, "w_sh leads the struct (16-byte aligned)");
 static_assert(offsetof(UmmaSmem, full) % 8 == 0, "mbarriers are 8-byte aligned");
@@ -177,7 +178,7 @@ template <int HI>
 __global__ void __launch_bounds__(kUmThreads, 1)
     index_score_umma_kernel(const __grid_constant__ CUtensorMap kmap, UmmaScoreArgs a) {
     constexpr int QG = 256 / HI;            // queries per CTA
-    constexpr int QW = 128 / HI;            // queries per epilogue warp
+    constexpr int QW = 64 / HI;             // queries per epilogue warp (64 columns)
     extern __shared__ uint8_t smem_um_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_um_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* qhi = base;
@@ -331,9 +332,12 @@ __global__ void __launch_bounds__(kUmThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue warps
-        const int quarter = warp & 3, half = warp >> 2;
+        // Warp w drains TMEM lanes 32(w%4).. (its 32 keys) and the 64
+        // columns 64(w/4).. (QW queries), releases the accumulator, then forms
+        // the scores without branches.
+        const int quarter = warp & 3, cg = warp >> 2;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        constexpr int LOGQ = QW == 32 ? 5 : QW == 16 ? 4 : 3;
+        constexpr int LOGQ = QW == 16 ? 4 : QW == 8 ? 3 : 2;
         const int my_q = lane >> (5 - LOGQ);                        // query slot this lane reduces
         const bool my_red = (lane & ((1 << (5 - LOGQ)) - 1)) == 0;  // one lane per slot writes
         int abuf = 0;
@@ -343,56 +347,62 @@ __global__ void __launch_bounds__(kUmThreads, 1)
             int vq[QW];   // visible blocks of each query of this warp in this pass (0: other sequence)
 #pragma unroll
             for (int qi = 0; qi < QW; ++qi) {
-                const int ql = half * QW + qi;
+                const int ql = cg * QW + qi;
                 vq[qi] = sm.seq_sh[ql] == seq ? sm.V_sh[ql] : 0;
             }
-            const int t_red = t0 + half * QW + my_q;
-            const int v_red = sm.seq_sh[half * QW + my_q] == seq ? sm.V_sh[half * QW + my_q] : 0;
+            const int t_red = t0 + cg * QW + my_q;
+            const int v_red = sm.seq_sh[cg * QW + my_q] == seq ? sm.V_sh[cg * QW + my_q] : 0;
+            float* const srow0 = a.scores + (int64_t)(t0 + cg * QW) * a.ld_scores;
             for (int j = 0; j < sm.ntiles[p]; ++j) {
                 const bool ok = mbar_wait_bounded(&sm.acc_full[abuf], aph, kUmWaitTries);
                 if (!ok && lane == 0) flag_status(a.status, kDevTimeout);
                 tc_fence_after();
-                uint32_t r[4][32];
-                const uint32_t col = tmem + lane_base + (uint32_t)(abuf * 256 + half * 128);
-                tmem_ld32(col, r[0], 0);
-                tmem_ld32(col, r[1], 32);
-                tmem_ld32(col, r[2], 64);
-                tmem_ld32(col, r[3], 96);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
+                const uint32_t col = tmem + lane_base + (uint32_t)(abuf * 256 + cg * 64);
+                const int g0 = j * kUmTile + quarter * 32;   // first key of this warp's 32-key group
+                const int key = g0 + lane;
+                float* srow = srow0 + key;
+                // two halves of 32 columns (QH queries each); the accumulator is
+                // released once the second half is in registers
+                constexpr int QH = QW / 2;
+                float sc[QW];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r[32];
+                    tmem_ld32(col, r, hh * 32);
+                    tmem_ld_wait();
+                    if (hh == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
+                    }
+                    if (!ok) continue;
+#pragma unroll
+                    for (int qh = 0; qh < QH; ++qh) {
+                        const int qi = hh * QH + qh;
+                        const float4* wp = reinterpret_cast<const float4*>(&sm.w_sh[(cg * QW + qi) * HI]);
+                        float s = 0.f;
+#pragma unroll
+                        for (int h4 = 0; h4 < HI / 4; ++h4) {
+                            const float4 wv = wp[h4];
+                            const int c = qh * HI + h4 * 4;
+                            s = fmaf(wv.x, fmaxf(__uint_as_float(r[c]), 0.f), s);
+                            s = fmaf(wv.y, fmaxf(__uint_as_float(r[c + 1]), 0.f), s);
+                            s = fmaf(wv.z, fmaxf(__uint_as_float(r[c + 2]), 0.f), s);
+                            s = fmaf(wv.w, fmaxf(__uint_as_float(r[c + 3]), 0.f), s);
+                        }
+                        const bool vis = key < vq[qi];
+                        if (vis) srow[(int64_t)qi * a.ld_scores] = s;
+                        sc[qi] = vis ? s : -INFINITY;
+                    }
+                }
                 if (++abuf == 2) {
                     abuf = 0;
                     aph ^= 1u;
                 }
                 if (!ok) continue;
-                const int g0 = j * kUmTile + quarter * 32;   // first key of this warp's 32-key group
-                const int key = g0 + lane;
-                // scores of the lane's key for the warp's queries (masked, no branches)
-                float sc[QW];
-#pragma unroll
-                for (int qi = 0; qi < QW; ++qi) {
-                    const float4* wp = reinterpret_cast<const float4*>(&sm.w_sh[(half * QW + qi) * HI]);
-                    float s = 0.f;
-#pragma unroll
-                    for (int h4 = 0; h4 < HI / 4; ++h4) {
-                        const float4 wv = wp[h4];
-                        const int c = qi * HI + h4 * 4;
-                        s = fmaf(wv.x, fmaxf(__uint_as_float(r[c >> 5][c & 31]), 0.f), s);
-                        s = fmaf(wv.y, fmaxf(__uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]), 0.f), s);
-                        s = fmaf(wv.z, fmaxf(__uint_as_float(r[(c + 2) >> 5][(c + 2) & 31]), 0.f), s);
-                        s = fmaf(wv.w, fmaxf(__uint_as_float(r[(c + 3) >> 5][(c + 3) & 31]), 0.f), s);
-                    }
-                    sc[qi] = s;
-                    if (key < vq[qi]) a.scores[(int64_t)(t0 + half * QW + qi) * a.ld_scores + key] = s;
-                }
                 if (a.hist) {
                     // maximum over the 32 keys of every query: halving exchange, after
                     // which lane l holds query slot l >> (5 - LOGQ)
-#pragma unroll
-                    for (int qi = 0; qi < QW; ++qi)
-                        if (!(key < vq[qi])) sc[qi] = -INFINITY;
                     int n = QW;
 #pragma unroll
                     for (int o = 16; o >= 1; o >>= 1) {
