@@ -312,7 +312,8 @@ def main():
         step_gbs = None
         tf_peak, tf_src = measured_tensor_peak()
         ach = fl["indexer"] / (k_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "kernel": "index_score_kernel", "achieved": round(ach, 2), "peak": tf_peak,
+        kname = "zero_state_kernel+index_score_umma_kernel"   # the stage timed by the events
+        roof = {"bound": "tensor", "kernel": kname, "achieved": round(ach, 2), "peak": tf_peak,
                 "unit": "TFLOP/s", "frac": round(ach / tf_peak, 4), "peak_source": tf_src, "traffic": None,
                 "algorithmic_flops_per_launch": fl["indexer"], "avg_launch_ms": round(k_ms, 5),
                 "step_flops": fl}
@@ -326,8 +327,15 @@ def main():
         else:
             kbytes, kname = ab["keys"], "index_score_kernel"
         ach = kbytes / (k_ms / 1e3) / 1e9
+        # DRAM bytes read + written per launch, from an ncu capture of this kernel
+        # (profiles/index_score_kernel_decode_b4_ctx1m.md: 4 of the 8 sequences,
+        # 139.96 MB; traffic grows with the sequences scored, so x2).  Only for
+        # the workload and key format it was measured on.
+        traffic = None
+        if args.workload == "csa_decode_1m" and args.kidx == "bf16" and not hca:
+            traffic = 279_916_544
         roof = {"bound": "hbm", "kernel": kname, "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(ach / peak, 4), "peak_source": peak_src, "traffic": None,
+                "frac": round(ach / peak, 4), "peak_source": peak_src, "traffic": traffic,
                 "algorithmic_bytes_per_launch": kbytes, "avg_launch_ms": round(k_ms, 5)}
 
     # end to end through the public API with pinned host buffers

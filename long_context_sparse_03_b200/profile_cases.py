@@ -1,0 +1,102 @@
+"""Small single-stage cases of the hot path, for profiling one kernel.
+
+    python -m long_context_sparse_03_b200.profile_cases score_decode [B]
+    python -m long_context_sparse_03_b200.profile_cases score_prefill [T]
+    python -m long_context_sparse_03_b200.profile_cases attend_prefill [T]
+
+Each case draws seeded inputs on the device, runs its libcsa call three
+times (a profiler skips the first and captures the second), checks the
+workspace status word, and prints the mean time of five further calls.
+
+* score_decode: csa_index_select for B queries, one per sequence of 262144
+  bf16 indexer keys (1M-token context, m = 4), Hi = 8, k = 1024 -- the
+  decode scoring kernel over B x 33.5 MB of keys.
+* score_prefill: csa_index_select for T consecutive query positions at the
+  end of one 139264-token sequence (34816 blocks), Hi = 8, k = 512 -- the
+  tensor-core (tcgen05) scoring kernel.
+* attend_prefill: csa_sparse_attend for T consecutive positions with 512
+  selected blocks each plus a 128-row window, H = 64 -- the fused
+  (one CTA per query) attention shape.
+"""
+from __future__ import annotations
+
+import sys
+
+import torch
+
+from . import csa
+
+
+def _time(fn, reps: int = 5) -> float:
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def _select_case(B: int, T: int, N: int, k: int, q_pos: torch.Tensor, q_seq: torch.Tensor, seed: int):
+    Hi, m = 8, 4
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    keys = torch.randn((B, N, 64), device="cuda", generator=g).to(torch.bfloat16)
+    q = torch.randn((T, Hi, 64), device="cuda", generator=g)
+    w = torch.randn((T, Hi), device="cuda", generator=g)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_index_workspace_size(T, 0, Hi, k, N))
+    return lambda: csa.csa_index_select(q, w, q_seq, q_pos, keys, m, N, k, idx, sc, ws), ws
+
+
+def score_decode(B: int = 4):
+    N = 262144
+    q_seq = torch.arange(B, dtype=torch.int32, device="cuda")
+    q_pos = torch.full((B,), N * 4 - 1, dtype=torch.int32, device="cuda")
+    return _select_case(B, B, N, 1024, q_pos, q_seq, 9)
+
+
+def score_prefill(T: int = 2048):
+    N = 34816
+    q_seq = torch.zeros(T, dtype=torch.int32, device="cuda")
+    q_pos = (N * 4 - T + torch.arange(T, device="cuda")).to(torch.int32)
+    return _select_case(1, T, N, 512, q_pos, q_seq, 5)
+
+
+def attend_prefill(T: int = 2048):
+    N, H, k, W, m = 34816, 64, 512, 128, 4
+    L = N * m
+    g = torch.Generator(device="cuda").manual_seed(3)
+    q = torch.randn((T, H, 128), device="cuda", generator=g).to(torch.bfloat16)
+    comp = torch.randn((1, N, 128), device="cuda", generator=g).to(torch.bfloat16)
+    raw = torch.randn((1, L, 128), device="cuda", generator=g).to(torch.bfloat16)
+    q_seq = torch.zeros(T, dtype=torch.int32, device="cuda")
+    q_pos = (L - T + torch.arange(T, device="cuda")).to(torch.int32)
+    # 512 distinct visible blocks per query (8 patterns repeated)
+    pat = torch.stack([torch.randperm(N - T // m, device="cuda", generator=g)[:k] for _ in range(8)]).to(torch.int32)
+    idx = pat.repeat((T + 7) // 8, 1)[:T].contiguous()
+    out = torch.empty((T, H, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, H), dtype=torch.float32, device="cuda")
+    ws = csa.Workspace(csa.csa_attend_workspace_size(T, H, k + W))
+    return lambda: csa.csa_sparse_attend(q, q_seq, q_pos, comp, raw, m, idx, W, 128 ** -0.5, out, lse, ws), ws
+
+
+CASES = {"score_decode": score_decode, "score_prefill": score_prefill, "attend_prefill": attend_prefill}
+
+
+def main(argv: list[str]) -> int:
+    if len(argv) < 1 or argv[0] not in CASES:
+        print(__doc__)
+        return 2
+    size = int(argv[1]) if len(argv) > 1 else None
+    fn, ws = CASES[argv[0]](size) if size else CASES[argv[0]]()
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ws.check()
+    print(f"{argv[0]} {size or ''} ms/call {_time(fn):.4f}", flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main(sys.argv[1:]))
