@@ -80,6 +80,10 @@ struct IndexLayout {
 // The scoring pass zeroes the selection state (hist, cnt, done: contiguous)
 // itself.  csa_index_query keeps u at the very end of whatever workspace it
 // is given.
+// Row stride of the workspace score matrix: a multiple of 4 floats, so every
+// row starts 16-byte aligned (the collect pass reads it 16 bytes at a time).
+int64_t score_ld(int max_blocks) { return ((int64_t)max_blocks + 3) & ~(int64_t)3; }
+
 IndexLayout index_layout(int T, int r, int Hi, int max_blocks) {
     IndexLayout L;
     size_t off = CSA_WS_HEADER_BYTES;
@@ -89,7 +93,7 @@ IndexLayout index_layout(int T, int r, int Hi, int max_blocks) {
     L.thr = L.done + (size_t)T * 4;
     off = up256(L.thr + (size_t)T * 4);
     L.scores = off;
-    off = up256(off + (size_t)T * max_blocks * 4);
+    off = up256(off + (size_t)T * score_ld(max_blocks) * 4);
     L.cand = off;
     off = up256(off + (size_t)T * cand_cap(max_blocks) * 8);
     L.q = off;
@@ -269,7 +273,7 @@ static csa_status stage_score(const char* who, const float* q, const float* w, c
     int n = 0;
     cudaError_t e = csa::launch_index_score(q, w, q_seq, q_pos, T, Hi, kidx, kidx_fmt, kidx_scale, kidx_seq_stride,
                                             scale_seq_stride, m, max_blocks, k,
-                                            reinterpret_cast<float*>(base + L.scores), max_blocks,
+                                            reinterpret_cast<float*>(base + L.scores), score_ld(max_blocks),
                                             reinterpret_cast<unsigned*>(base + L.hist),
                                             reinterpret_cast<unsigned*>(base + L.cnt),
                                             reinterpret_cast<unsigned*>(base + L.done),
@@ -286,7 +290,7 @@ static csa_status stage_merge(const char* who, const int32_t* q_pos, int T, int 
     char* base = (char*)ws;
     int n = 0;
     cudaError_t e = csa::launch_index_select_tail(
-        reinterpret_cast<const float*>(base + L.scores), max_blocks, reinterpret_cast<const unsigned*>(base + L.thr),
+        reinterpret_cast<const float*>(base + L.scores), score_ld(max_blocks), reinterpret_cast<const unsigned*>(base + L.thr),
         q_pos, T, m, max_blocks, k, reinterpret_cast<uint64_t*>(base + L.cand), cand_cap(max_blocks),
         reinterpret_cast<unsigned*>(base + L.cnt), out_idx, out_score, stream, &n);
     count(n);

@@ -646,7 +646,9 @@ __global__ void __launch_bounds__(kScoreCta, 2) index_score_kernel(ScoreArgs a) 
 
 // ---------------------------------------------------------------- collect
 // grid (ceil(max_blocks / kCollectKeys), T), 256 threads: append every score
-// whose key reaches the query's threshold to its candidate list.
+// whose key reaches the query's threshold to its candidate list.  Rows of the
+// score matrix start 16-byte aligned (ld_scores a multiple of 4), so each
+// thread reads its 16 scores as four 16-byte loads, all in flight at once.
 __global__ void __launch_bounds__(256) collect_kernel(const float* __restrict__ scores, int64_t ld_scores,
                                                       const unsigned* __restrict__ thr_t, const int* __restrict__ q_pos,
                                                       int m, int max_blocks, uint64_t* __restrict__ cand,
@@ -661,20 +663,24 @@ __global__ void __launch_bounds__(256) collect_kernel(const float* __restrict__ 
     uint64_t* crow = cand + (int64_t)t * cand_cap;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int j1 = min(j0 + kCollectKeys, V);
-    constexpr int PER = kCollectKeys / 256;
+    constexpr int P4 = kCollectKeys / 1024;   // 16-byte loads per thread
     __shared__ unsigned wcount[8], wbase[8];
-    float sv[PER];
+    float4 sv[P4];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {   // all loads in flight before any use
-        const int j = j0 + e * 256 + threadIdx.x;
-        sv[e] = j < j1 ? srow[j] : 0.f;
+    for (int e = 0; e < P4; ++e) {   // j is a multiple of 4 below ld_scores: the load stays in the row
+        const int j = j0 + e * 1024 + threadIdx.x * 4;
+        sv[e] = j < j1 ? __ldcs(reinterpret_cast<const float4*>(srow + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    unsigned bal[PER], mine = 0;
+    unsigned bal[P4][4], mine = 0;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-        const int j = j0 + e * 256 + threadIdx.x;
-        bal[e] = __ballot_sync(0xffffffffu, j < j1 && score_key(sv[e]) >= thr);
-        mine += __popc(bal[e]);
+    for (int e = 0; e < P4; ++e) {
+        const int j = j0 + e * 1024 + threadIdx.x * 4;
+        const float x[4] = {sv[e].x, sv[e].y, sv[e].z, sv[e].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            bal[e][c] = __ballot_sync(0xffffffffu, j + c < j1 && score_key(x[c]) >= thr);
+            mine += __popc(bal[e][c]);
+        }
     }
     if (lane == 0) wcount[warp] = mine;
     __syncthreads();
@@ -689,13 +695,16 @@ __global__ void __launch_bounds__(256) collect_kernel(const float* __restrict__ 
     }
     __syncthreads();
     unsigned pos = wbase[warp];
+    const unsigned below = (1u << lane) - 1u;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-        if (bal[e] >> lane & 1u) {
-            const int j = j0 + e * 256 + threadIdx.x;
-            crow[pos + __popc(bal[e] & ((1u << lane) - 1u))] = make_cand(sv[e], j);
+    for (int e = 0; e < P4; ++e) {
+        const int j = j0 + e * 1024 + threadIdx.x * 4;
+        const float x[4] = {sv[e].x, sv[e].y, sv[e].z, sv[e].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (bal[e][c] >> lane & 1u) crow[pos + __popc(bal[e][c] & below)] = make_cand(x[c], j + c);
+            pos += __popc(bal[e][c]);
         }
-        pos += __popc(bal[e]);
     }
     griddep_trigger();
 }
@@ -719,6 +728,7 @@ __device__ __forceinline__ void write_out(int* out_idx, float* out_score, int64_
 
 // Rank the n distinct nonzero keys v[0..n) (shared) and write those of rank
 // < k.  Scratch: bucket[n] (shared), hist/start[kRankBins] (shared).
+template <int NTH>
 __device__ void rank_write(const uint64_t* v, int n, int k, uint64_t* bucket, unsigned* hist, unsigned* start,
                            int* out_idx, float* out_score, int64_t out_off) {
     __shared__ unsigned long long red[2];
@@ -744,7 +754,7 @@ __device__ void rank_write(const uint64_t* v, int n, int k, uint64_t* bucket, un
     for (int i = tid; i < n; i += nth) atomicAdd(&hist[(unsigned)(v[i] >> sh) & (kRankBins - 1)], 1u);
     __syncthreads();
     // start[b] = number of keys in buckets above b (exclusive scan from the top)
-    constexpr int per = kRankBins / kRankThreads;   // 2
+    constexpr int per = kRankBins / NTH;   // bins per thread
     unsigned c[per], tot = 0;
 #pragma unroll
     for (int e = 0; e < per; ++e) {
@@ -787,11 +797,14 @@ __device__ void rank_write(const uint64_t* v, int n, int k, uint64_t* bucket, un
 }
 
 // grid (T), kRankThreads threads.
-__global__ void __launch_bounds__(kRankThreads) rank_kernel(const uint64_t* __restrict__ cand, int64_t cand_cap,
-                                                          const unsigned* __restrict__ cnt, int k,
-                                                          int* __restrict__ out_idx, float* __restrict__ out_score) {
-    extern __shared__ __align__(16) uint64_t v[];   // [kRankCap] list, [kRankCap] buckets
-    uint64_t* bucket = v + kRankCap;
+// NTH threads; CAP candidates ranked from shared memory (longer lists are
+// first cut to k by the radix select).
+template <int NTH, int CAP>
+__global__ void __launch_bounds__(NTH) rank_kernel(const uint64_t* __restrict__ cand, int64_t cand_cap,
+                                                   const unsigned* __restrict__ cnt, int k,
+                                                   int* __restrict__ out_idx, float* __restrict__ out_score) {
+    extern __shared__ __align__(16) uint64_t v[];   // [CAP] list, [CAP] buckets
+    uint64_t* bucket = v + CAP;
     __shared__ unsigned hist[kRankBins];
     __shared__ unsigned start[kRankBins];
     __shared__ int misc[8];
@@ -804,7 +817,7 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const uint64_t* __re
         if (out_score) out_score[(int64_t)t * k + i] = __int_as_float(0x7fc00000);
     }
     int ns = n;
-    if (n <= kRankCap) {
+    if (n <= CAP) {
         // stage with cp.async (every 16-byte piece in flight); an odd last
         // element is zero-filled past the end
         for (int i = 2 * threadIdx.x; i < n; i += 2 * blockDim.x) cp_async16(v + i, src + i, i + 1 < n ? 16 : 8);
@@ -824,7 +837,7 @@ __global__ void __launch_bounds__(kRankThreads) rank_kernel(const uint64_t* __re
         __syncthreads();
         ns = misc[4];
     }
-    rank_write(v, ns, k, bucket, hist, start, out_idx, out_score, (int64_t)t * k);
+    rank_write<NTH>(v, ns, k, bucket, hist, start, out_idx, out_score, (int64_t)t * k);
     griddep_trigger();
 }
 
@@ -837,6 +850,8 @@ cudaError_t launch_index_score_umma(const float* q, const float* w, const int* q
 
 static int g_sm_count[64];
 static int g_score_occ[64][2][2];
+
+static int sm_count_current() { return current_sm_count(); }
 
 static int sm_count(int dev) {
     if (dev < 0 || dev >= 64) return 148;
@@ -920,11 +935,18 @@ cudaError_t launch_index_select_tail(const float* scores, int64_t ld_scores, con
     cudaError_t e = launch_pdl(collect_kernel, g1, dim3(256), 0, stream, scores, ld_scores, thr, q_pos, m, max_blocks,
                                cand, cand_cap, cnt);
     if (e != cudaSuccess) return e;
-    const size_t rank_smem = (size_t)2 * kRankCap * 8;
-    e = cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(rank_kernel, dim3(T), dim3(kRankThreads), rank_smem, stream, (const uint64_t*)cand, cand_cap,
-                   (const unsigned*)cnt, k, out_idx, out_score);
+    // Few queries: one 1024-thread CTA per query with room for 8192
+    // candidates.  Many queries (prefill): 512 threads and 4096 candidates,
+    // so two CTAs share an SM.
+    auto go = [&](auto kern, int threads, int cap) {
+        const size_t smem = (size_t)2 * cap * 8;
+        cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e2 != cudaSuccess) return e2;
+        return launch_pdl(kern, dim3(T), dim3(threads), smem, stream, (const uint64_t*)cand, cand_cap,
+                          (const unsigned*)cnt, k, out_idx, out_score);
+    };
+    if (T >= 2 * sm_count_current()) e = go(rank_kernel<512, 4096>, 512, 4096);
+    else e = go(rank_kernel<kRankThreads, kRankCap>, kRankThreads, kRankCap);
     if (e != cudaSuccess) return e;
     *launches += 2;
     return e;
