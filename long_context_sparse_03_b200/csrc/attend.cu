@@ -128,14 +128,17 @@ __global__ void __launch_bounds__(NW * 32, NW <= 4 ? 3 : 1)
     const int gb_hi = FUSED ? nb_total : min(nb_total, gb_lo + bps);
 
     // issue the gather of row block `gb` (list positions gb*64 ..) into buffer `buf`
+    // (a pair of threads per row: one row lookup, then 8 x 16 bytes each)
     auto gather = [&](int gb, int buf) {
-        for (int i = threadIdx.x; i < kRowBlock * 16; i += NW * 32) {
-            const int r = i >> 4, c = i & 15;
+        for (int i = threadIdx.x; i < kRowBlock * 2; i += NW * 32) {
+            const int r = i >> 1, c0 = (i & 1) * 8;
             const int pos = gb * kRowBlock + r;
             const bf16* src = pos < total ? row_ptr(a, t, b, p, V, nsel, pos) : nullptr;
-            cp_async16(&rows_sh[buf][r * kRowStride + c * 8], src ? (const void*)(src + c * 8) : (const void*)a.raw,
-                       src ? 16 : 0);
-            if (c == 0) valid_sh[buf][r] = src != nullptr;
+#pragma unroll
+            for (int c = c0; c < c0 + 8; ++c)
+                cp_async16(&rows_sh[buf][r * kRowStride + c * 8],
+                           src ? (const void*)(src + c * 8) : (const void*)a.raw, src ? 16 : 0);
+            if (c0 == 0) valid_sh[buf][r] = src != nullptr;
         }
         cp_async_commit();
     };
