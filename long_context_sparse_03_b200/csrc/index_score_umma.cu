@@ -8,8 +8,9 @@
 // the key cache (M = keys) with the stacked query heads (N = queries x Hi,
 // K = 64 channels), followed by a per-query epilogue (ReLU, weighted head sum).
 //
-// One CTA owns QG = 256 / Hi consecutive queries (N = 256 columns) for the
-// whole key range, so its epilogue sees every score of those queries:
+// A CTA owns QG = 256 / Hi consecutive queries (N = 256 columns) and one of
+// P pieces of their key range (P chosen so that the grid fills its last
+// wave; the last piece to finish turns the histograms into thresholds):
 //   * warp 16 (one lane) streams 128-key tiles of the cache into a 4-stage
 //     ring with 3-D TMA tensor copies (128-byte swizzle, the canonical K-major
 //     operand layout of the tensor core);
@@ -60,7 +61,9 @@ struct UmmaScoreArgs {
     int64_t ld_scores;
     unsigned* hist;       // [T][2048]
     unsigned* thr;        // [T]
+    unsigned* done;       // [T]: pieces finished, counted at the group's first query
     unsigned* status;
+    int pieces;           // CTAs sharing one query group's key tiles
 };
 
 struct UmmaSmem {
@@ -71,6 +74,8 @@ struct UmmaSmem {
     int seqs[64], ntiles[64];
     int V_sh[64], seq_sh[64];
     int Vp[64];   // visible blocks per query in the current pass (0: another sequence)
+    int lo, hi;   // this CTA's piece of the group's flattened (pass, tile) sequence
+    int last;     // this CTA finished the group's last piece
 };
 static_assert(offsetof(UmmaSmem, w_sh) == 0, "w_sh leads the struct (16-byte aligned)");
 static_assert(offsetof(UmmaSmem, full) % 8 == 0, "mbarriers are 8-byte aligned");
@@ -134,19 +139,13 @@ __device__ __forceinline__ void tma_load_keys(void* dst, const CUtensorMap* map,
 // top reaches k walks its bins.
 __device__ unsigned warp_threshold_bin(const unsigned* gh, int k) {
     const int lane = threadIdx.x & 31;
-    const unsigned* mine = gh + kUmHistBins - 64 * (lane + 1);
-    unsigned c[64];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(mine) + i);
-        c[4 * i] = v.x;
-        c[4 * i + 1] = v.y;
-        c[4 * i + 2] = v.z;
-        c[4 * i + 3] = v.w;
-    }
+    const uint4* mine = reinterpret_cast<const uint4*>(gh + kUmHistBins - 64 * (lane + 1));
     unsigned s = 0;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) s += c[i];
+#pragma unroll 4
+    for (int i = 0; i < 16; ++i) {
+        const uint4 v = __ldcg(mine + i);
+        s += v.x + v.y + v.z + v.w;
+    }
     unsigned incl = s;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -159,14 +158,21 @@ __device__ unsigned warp_threshold_bin(const unsigned* gh, int k) {
     if (hit) {
         const int src = __ffs(hit) - 1;
         unsigned bin = 0;
-        if (lane == src) {
+        if (lane == src) {   // walk this lane's bins from its top one down
             unsigned run = excl;
-            for (int i = 63; i >= 0; --i) {   // from the lane's top bin down
-                run += c[i];
-                if (run >= (unsigned)k) {
-                    bin = (unsigned)(kUmHistBins - 64 * (lane + 1) + i);
-                    break;
+            for (int i = 15; i >= 0; --i) {
+                const uint4 v = __ldcg(mine + i);
+                const unsigned c[4] = {v.w, v.z, v.y, v.x};
+                bool found = false;
+                for (int e = 0; e < 4; ++e) {
+                    run += c[e];
+                    if (run >= (unsigned)k) {
+                        bin = (unsigned)(kUmHistBins - 64 * (lane + 1) + 4 * i + (3 - e));
+                        found = true;
+                        break;
+                    }
                 }
+                if (found) break;
             }
         }
         b = __shfl_sync(0xffffffffu, bin, src);
@@ -186,7 +192,8 @@ __global__ void __launch_bounds__(kUmThreads, 1)
     uint8_t* kst = base + 2 * kUmQBytes;
     UmmaSmem& sm = *reinterpret_cast<UmmaSmem*>(kst + kUmStages * kUmTileBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = blockIdx.x * QG;
+    const int piece = blockIdx.x % a.pieces;
+    const int t0 = (blockIdx.x / a.pieces) * QG;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kUmStages; ++s) {
@@ -270,10 +277,17 @@ __global__ void __launch_bounds__(kUmThreads, 1)
         }
         sm.nseq = ns;
         sm.ntiles_total = tot;
+        sm.lo = (int)((int64_t)tot * piece / a.pieces);
+        sm.hi = (int)((int64_t)tot * (piece + 1) / a.pieces);
     }
     __syncthreads();
     const uint32_t tmem = sm.tmem_base;
-    const int nseq = sm.nseq, ntot = sm.ntiles_total;
+    const int nseq = sm.nseq;
+    const int ntot = sm.hi - sm.lo;   // tiles of this CTA
+    // (pass, tile) of flattened index sm.lo: the piece starts there and runs
+    // through ntot tiles of the passes in order
+    int p0 = 0, j0 = sm.lo;
+    while (p0 < nseq && j0 >= sm.ntiles[p0]) j0 -= sm.ntiles[p0++];
 
     if (warp == kUmEpiWarps) {
         // ------------------------------------------------ TMA producer
@@ -281,8 +295,9 @@ __global__ void __launch_bounds__(kUmThreads, 1)
             int slot = 0;
             unsigned ph = 0;
             int it = 0;
-            for (int p = 0; p < nseq; ++p) {
-                for (int j = 0; j < sm.ntiles[p]; ++j, ++it) {
+            for (int p = p0; p < nseq && it < ntot; ++p) {
+                const int jb = p == p0 ? j0 : 0, je = min(sm.ntiles[p], jb + (ntot - it));
+                for (int j = jb; j < je; ++j, ++it) {
                     if (it >= kUmStages && !mbar_wait_bounded(&sm.empty[slot], ph ^ 1u, kUmWaitTries))
                         flag_status(a.status, kDevTimeout);
                     mbar_arrive_expect_tx(&sm.full[slot], kUmTileBytes);
@@ -342,94 +357,104 @@ __global__ void __launch_bounds__(kUmThreads, 1)
         const bool my_red = (lane & ((1 << (5 - LOGQ)) - 1)) == 0;  // one lane per slot writes
         int abuf = 0;
         unsigned aph = 0;
-        for (int p = 0; p < nseq; ++p) {
+        const int t_red = t0 + cg * QW + my_q;
+        float* const srow0 = a.scores + (int64_t)(t0 + cg * QW) * a.ld_scores;
+        int vq[QW];   // visible blocks of each query of this warp in the current pass (0: other sequence)
+        int left = ntot;
+        for (int p = p0; p < nseq && left > 0; ++p) {
             const int seq = sm.seqs[p];
-            int vq[QW];   // visible blocks of each query of this warp in this pass (0: other sequence)
 #pragma unroll
             for (int qi = 0; qi < QW; ++qi) {
                 const int ql = cg * QW + qi;
                 vq[qi] = sm.seq_sh[ql] == seq ? sm.V_sh[ql] : 0;
             }
-            const int t_red = t0 + cg * QW + my_q;
             const int v_red = sm.seq_sh[cg * QW + my_q] == seq ? sm.V_sh[cg * QW + my_q] : 0;
-            float* const srow0 = a.scores + (int64_t)(t0 + cg * QW) * a.ld_scores;
-            for (int j = 0; j < sm.ntiles[p]; ++j) {
-                const bool ok = mbar_wait_bounded(&sm.acc_full[abuf], aph, kUmWaitTries);
-                if (!ok && lane == 0) flag_status(a.status, kDevTimeout);
-                tc_fence_after();
-                const uint32_t col = tmem + lane_base + (uint32_t)(abuf * 256 + cg * 64);
-                const int g0 = j * kUmTile + quarter * 32;   // first key of this warp's 32-key group
-                const int key = g0 + lane;
-                float* srow = srow0 + key;
-                // two halves of 32 columns (QH queries each); the accumulator is
-                // released once the second half is in registers
-                constexpr int QH = QW / 2;
-                float sc[QW];
+            const int jb = p == p0 ? j0 : 0, je = min(sm.ntiles[p], jb + left);
+            left -= je - jb;
+            for (int j = jb; j < je; ++j) {
+            const bool ok = mbar_wait_bounded(&sm.acc_full[abuf], aph, kUmWaitTries);
+            if (!ok && lane == 0) flag_status(a.status, kDevTimeout);
+            tc_fence_after();
+            const uint32_t col = tmem + lane_base + (uint32_t)(abuf * 256 + cg * 64);
+            const int g0 = j * kUmTile + quarter * 32;   // first key of this warp's 32-key group
+            const int key = g0 + lane;
+            float* srow = srow0 + key;
+            // two halves of 32 columns (QH queries each); the accumulator is
+            // released once the second half is in registers
+            constexpr int QH = QW / 2;
+            float sc[QW];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t r[32];
-                    tmem_ld32(col, r, hh * 32);
-                    tmem_ld_wait();
-                    if (hh == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
-                    }
-                    if (!ok) continue;
-#pragma unroll
-                    for (int qh = 0; qh < QH; ++qh) {
-                        const int qi = hh * QH + qh;
-                        const float4* wp = reinterpret_cast<const float4*>(&sm.w_sh[(cg * QW + qi) * HI]);
-                        float s = 0.f;
-#pragma unroll
-                        for (int h4 = 0; h4 < HI / 4; ++h4) {
-                            const float4 wv = wp[h4];
-                            const int c = qh * HI + h4 * 4;
-                            s = fmaf(wv.x, fmaxf(__uint_as_float(r[c]), 0.f), s);
-                            s = fmaf(wv.y, fmaxf(__uint_as_float(r[c + 1]), 0.f), s);
-                            s = fmaf(wv.z, fmaxf(__uint_as_float(r[c + 2]), 0.f), s);
-                            s = fmaf(wv.w, fmaxf(__uint_as_float(r[c + 3]), 0.f), s);
-                        }
-                        const bool vis = key < vq[qi];
-                        if (vis) srow[(int64_t)qi * a.ld_scores] = s;
-                        sc[qi] = vis ? s : -INFINITY;
-                    }
-                }
-                if (++abuf == 2) {
-                    abuf = 0;
-                    aph ^= 1u;
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t r[32];
+                tmem_ld32(col, r, hh * 32);
+                tmem_ld_wait();
+                if (hh == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
                 }
                 if (!ok) continue;
-                if (a.hist) {
-                    // maximum over the 32 keys of every query: halving exchange, after
-                    // which lane l holds query slot l >> (5 - LOGQ)
-                    int n = QW;
 #pragma unroll
-                    for (int o = 16; o >= 1; o >>= 1) {
-                        if (n > 1) {
-                            const bool upper = (lane & o) != 0;
+                for (int qh = 0; qh < QH; ++qh) {
+                    const int qi = hh * QH + qh;
+                    const float4* wp = reinterpret_cast<const float4*>(&sm.w_sh[(cg * QW + qi) * HI]);
+                    float s = 0.f;
 #pragma unroll
-                            for (int i = 0; i < QW / 2; ++i) {
-                                if (i < n / 2) {
-                                    const float send = upper ? sc[i] : sc[i + n / 2];
-                                    const float keep = upper ? sc[i + n / 2] : sc[i];
-                                    sc[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
-                                }
-                            }
-                            n >>= 1;
-                        } else {
-                            sc[0] = fmaxf(sc[0], __shfl_xor_sync(0xffffffffu, sc[0], o));
-                        }
+                    for (int h4 = 0; h4 < HI / 4; ++h4) {
+                        const float4 wv = wp[h4];
+                        const int c = qh * HI + h4 * 4;
+                        s = fmaf(wv.x, fmaxf(__uint_as_float(r[c]), 0.f), s);
+                        s = fmaf(wv.y, fmaxf(__uint_as_float(r[c + 1]), 0.f), s);
+                        s = fmaf(wv.z, fmaxf(__uint_as_float(r[c + 2]), 0.f), s);
+                        s = fmaf(wv.w, fmaxf(__uint_as_float(r[c + 3]), 0.f), s);
                     }
-                    if (my_red && g0 < v_red)
-                        atomicAdd(&a.hist[(int64_t)t_red * kUmHistBins + (score_key(sc[0]) >> kUmHistShift)], 1u);
+                    const bool vis = key < vq[qi];
+                    if (vis) srow[(int64_t)qi * a.ld_scores] = s;
+                    sc[qi] = vis ? s : -INFINITY;
                 }
+            }
+            if (++abuf == 2) {
+                abuf = 0;
+                aph ^= 1u;
+            }
+            if (!ok) continue;
+            if (a.hist) {
+                // maximum over the 32 keys of every query: halving exchange, after
+                // which lane l holds query slot l >> (5 - LOGQ)
+                int n = QW;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    if (n > 1) {
+                        const bool upper = (lane & o) != 0;
+#pragma unroll
+                        for (int i = 0; i < QW / 2; ++i) {
+                            if (i < n / 2) {
+                                const float send = upper ? sc[i] : sc[i + n / 2];
+                                const float keep = upper ? sc[i + n / 2] : sc[i];
+                                sc[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, o));
+                            }
+                        }
+                        n >>= 1;
+                    } else {
+                        sc[0] = fmaxf(sc[0], __shfl_xor_sync(0xffffffffu, sc[0], o));
+                    }
+                }
+                if (my_red && g0 < v_red)
+                    atomicAdd(&a.hist[(int64_t)t_red * kUmHistBins + (score_key(sc[0]) >> kUmHistShift)], 1u);
+            }
             }
         }
         // every histogram count of this CTA's queries is in: threshold keys
         __threadfence();
         named_sync(1, kUmEpiWarps * 32);
-        for (int ql = warp; ql < QG && a.hist; ql += kUmEpiWarps) {
+        bool finish = a.hist != nullptr;
+        if (finish && a.pieces > 1) {   // only the group's last piece turns histograms into thresholds
+            if (threadIdx.x == 0) sm.last = atomicAdd(&a.done[t0], 1u) == (unsigned)(a.pieces - 1);
+            named_sync(1, kUmEpiWarps * 32);
+            finish = sm.last != 0;
+            if (finish) __threadfence();
+        }
+        for (int ql = warp; ql < QG && finish; ql += kUmEpiWarps) {
             const int t = t0 + ql;
             if (t >= a.T) break;
             const unsigned b = warp_threshold_bin(a.hist + (int64_t)t * kUmHistBins, a.k);
@@ -473,8 +498,8 @@ bool index_score_umma_applies(int T, int Hi, int fmt, const float* q, const void
 
 cudaError_t launch_index_score_umma(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
                                     const void* kidx, int64_t kstride_bytes, int m, int max_blocks, int k,
-                                    float* scores, int64_t ld_scores, unsigned* hist, unsigned* thr, unsigned* status,
-                                    cudaStream_t stream) {
+                                    float* scores, int64_t ld_scores, unsigned* hist, unsigned* thr, unsigned* done,
+                                    unsigned* status, cudaStream_t stream) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap map;
@@ -501,12 +526,32 @@ cudaError_t launch_index_score_umma(const float* q, const float* w, const int* q
     a.ld_scores = ld_scores;
     a.hist = hist;
     a.thr = thr;
+    a.done = done;
     a.status = status;
+    // Pieces per query group: split a group's key tiles over P CTAs when that
+    // fills the SMs markedly better (each CTA has a fixed cost -- q staging,
+    // TMEM allocation, pipeline fill -- which measured as large as the gain
+    // from only evening out a last wave); a piece keeps at least 16 tiles.
+    const int qg_hi = 256 / Hi;
+    const int64_t G = (T + qg_hi - 1) / qg_hi, S = current_sm_count();
+    const int max_tiles = (max_blocks + kUmTile - 1) / kUmTile;
+    int P = 1;
+    double best = (double)G / (double)(((G + S - 1) / S) * S);
+    for (int pp = 2; pp <= 4 && max_tiles / pp >= 16; ++pp) {
+        const int64_t n = G * pp;
+        const double eff = (double)n / (double)(((n + S - 1) / S) * S);
+        if (eff > 1.2 * best) {
+            best = eff;
+            P = pp;
+        }
+    }
+    if (hist && !done) P = 1;
+    a.pieces = P;
     const size_t smem = umma_smem_bytes();
     auto go = [&](auto kern, int qg) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(kern, dim3((unsigned)((T + qg - 1) / qg)), dim3(kUmThreads), smem, stream, map, a);
+        return launch_pdl(kern, dim3((unsigned)(((T + qg - 1) / qg) * P)), dim3(kUmThreads), smem, stream, map, a);
     };
     if (Hi == 4) return go(index_score_umma_kernel<4>, 64);
     if (Hi == 8) return go(index_score_umma_kernel<8>, 32);

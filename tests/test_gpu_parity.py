@@ -159,9 +159,11 @@ def _keys_f64(oracle, keys, kscale, fmt):
 
 
 # T >= 256 with bf16 keys and Hi in {4, 8, 16} runs the tensor-core (tcgen05)
-# scoring kernel; the queries of those cases mix two sequences.
+# scoring kernel; the queries of those cases mix two sequences, and with
+# 9000 blocks each query group's key range is split over several CTAs.
 @pytest.mark.parametrize("fmt,Hi,N,T", [(0, 8, 5000, 6), (1, 8, 5000, 6), (0, 4, 1024, 1), (0, 16, 3000, 4),
-                                        (1, 3, 2100, 3), (0, 8, 3000, 300), (0, 4, 2000, 260), (0, 16, 1500, 256)])
+                                        (1, 3, 2100, 3), (0, 8, 3000, 300), (0, 4, 2000, 260), (0, 16, 1500, 256),
+                                        (0, 8, 9000, 280)])
 def test_index_scores(oracle, fmt, Hi, N, T):
     rng = np.random.default_rng(fmt * 10 + Hi + N)
     m = 4
@@ -183,7 +185,8 @@ def test_index_scores(oracle, fmt, Hi, N, T):
     (0, 8, 5000, 6, 64, False, False), (0, 8, 9000, 3, 512, False, False), (1, 8, 9000, 3, 512, False, False),
     (0, 4, 1024, 1, 64, False, False), (0, 8, 3000, 4, 2048, False, False), (0, 8, 2500, 5, 1, False, False),
     (0, 8, 4000, 4, 100, True, False), (0, 8, 4000, 4, 300, False, True), (1, 16, 20000, 2, 1024, False, False),
-    (0, 8, 3000, 300, 256, False, False), (0, 8, 4000, 260, 100, True, False), (0, 16, 2500, 300, 512, False, True)])
+    (0, 8, 3000, 300, 256, False, False), (0, 8, 4000, 260, 100, True, False), (0, 16, 2500, 300, 512, False, True),
+    (0, 8, 9000, 300, 512, False, False), (0, 4, 9000, 270, 64, True, False)])
 def test_index_select(oracle, fmt, Hi, N, T, k, ties, neg):
     rng = np.random.default_rng(1000 + fmt + Hi + N + k)
     m = 4
