@@ -184,6 +184,18 @@ CSA_API csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
  * fp32 [B][scale_seq_stride] (CSA_FMT_FP8E4M3).  Uses the same scoring
  * arithmetic as csa_index_select.
  */
+/*
+ * Scoring kernels (csa_index_scores, csa_index_select, csa_index_stage_score,
+ * csa_index_topk).  With T >= 256 queries, bf16 keys and Hi in {4, 8, 16}
+ * the scores come from a tensor-core (tcgen05) kernel that reads the key
+ * cache in whole 128-row tiles: each sequence's cache must then hold
+ * max_blocks rows (rows past a query's V are read and ignored; q_seq values
+ * must be below CSA_MAX_T).  Fewer queries use the streaming decode kernel,
+ * which reads only visible rows.  The two kernels group the products
+ * differently, so a query's scores may differ in the last bits between a
+ * call below and a call at or above T = 256 (both within the stated score
+ * tolerance); within either regime results do not depend on the batch.
+ */
 CSA_API csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq,
                             const int32_t* q_pos, int T, int Hi,
                             const void* kidx, int kidx_fmt, const float* kidx_scale,
