@@ -46,7 +46,10 @@
  *     the token's own raw row is already in the raw cache.
  *   - Results are deterministic and batch-invariant: a query's outputs are
  *     bitwise the same whatever other queries share the call, and across
- *     runs (fixed split sizes, no floating-point atomics).
+ *     runs (fixed split sizes, no floating-point atomics).  One exception:
+ *     the indexer scores come from a different kernel from T = 256 queries
+ *     on (see section 2), so they can differ in the last bits across that
+ *     boundary.
  *   - Device-side anomalies (an out-of-range block index) never trap: the
  *     offending entry is skipped and a bit is set in a status word at the
  *     start of the workspace; csa_status_check() reads and clears it.
