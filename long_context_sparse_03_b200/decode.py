@@ -121,25 +121,50 @@ class CsaDecoder:
         self.attend()
         return self.out
 
-    def step_host(self, h_host, q_host, kv_row_host, ki_row_host, out_host):
-        """The same step from pinned host buffers: copy this step's inputs
-        (hidden states, attention queries, the new token's raw rows) to the
-        device, run the step, copy the attention output back."""
+    # -- the step from one packed pinned host buffer -------------------
+    def packed_layout(self) -> dict:
+        """Byte layout of one step's inputs in a single buffer: name ->
+        (offset, shape, dtype), every section 256-byte aligned.  Sections:
+        hidden states h [T][D], attention queries q [T][H][128], and the new
+        token's raw latent and indexer-key rows [T][128], [T][64]."""
+        i, w = self.inp, self.w
+        secs = [("h", tuple(i.h.shape), i.h.dtype), ("q", tuple(i.q.shape), i.q.dtype),
+                ("kv_row", (w.B, 128), i.raw_kv.dtype), ("ki_row", (w.B, 64), i.raw_ki.dtype)]
+        lay, off = {}, 0
+        for name, shape, dt in secs:
+            n = 1
+            for x in shape:
+                n *= x
+            lay[name] = (off, shape, dt)
+            off = (off + n * torch.tensor([], dtype=dt).element_size() + 255) // 256 * 256
+        lay["_bytes"] = off
+        return lay
+
+    def step_packed(self, in_host: torch.Tensor, out_host: torch.Tensor):
+        """The step with all its inputs in one pinned uint8 buffer laid out by
+        packed_layout(): one host-to-device copy, the step (reading h and q
+        straight from the staged copy), one device-to-host copy of the output."""
         i = self.inp
-        if not hasattr(self, "_rows"):
+        if not hasattr(self, "_stage"):
+            lay = self.packed_layout()
             dev = i.raw_kv.device
+            self._stage = torch.empty(lay["_bytes"], dtype=torch.uint8, device=dev)
+
+            def view(name):
+                off, shape, dt = lay[name]
+                n = 1
+                for x in shape:
+                    n *= x
+                nb = n * torch.tensor([], dtype=dt).element_size()
+                return self._stage[off:off + nb].view(dt).view(shape)
+            i.h, i.q = view("h"), view("q")
+            self._kv_new, self._ki_new = view("kv_row"), view("ki_row")
             self._pos = (i.lens.long() - 1).to(dev)
             self._bidx = torch.arange(self.w.B, device=dev)
-            self._kv_rows = torch.empty(kv_row_host.shape, dtype=kv_row_host.dtype, device=dev)
-            self._ki_rows = torch.empty(ki_row_host.shape, dtype=ki_row_host.dtype, device=dev)
-            self._rows = True
         with torch.cuda.stream(self._s()):
-            i.h.copy_(h_host, non_blocking=True)
-            i.q.copy_(q_host, non_blocking=True)
-            self._kv_rows.copy_(kv_row_host, non_blocking=True)
-            self._ki_rows.copy_(ki_row_host, non_blocking=True)
-            i.raw_kv.index_put_((self._bidx, self._pos), self._kv_rows)
-            i.raw_ki.index_put_((self._bidx, self._pos), self._ki_rows)
+            self._stage.copy_(in_host, non_blocking=True)
+            i.raw_kv.index_put_((self._bidx, self._pos), self._kv_new)
+            i.raw_ki.index_put_((self._bidx, self._pos), self._ki_new)
         self.step()
         with torch.cuda.stream(self._s()):
             out_host.copy_(self.out, non_blocking=True)

@@ -450,3 +450,33 @@ def test_index_select_all_ties(oracle, fmt):
         assert np.array_equal(gi[t, :n], np.arange(n)), t
         assert (gi[t, n:] == -1).all()
         assert (sc[t, :n].cpu().numpy() == 0).all()
+
+
+def test_decode_step_packed_inputs_match_device_step():
+    """The end-to-end step (one pinned buffer -> one host-to-device copy ->
+    the step -> the output copied back) returns exactly the device step's
+    output for the same inputs."""
+    from long_context_sparse_03_b200 import workloads as wl
+    from long_context_sparse_03_b200.decode import CsaDecoder
+    w = wl.scaled(wl.CSA_DECODE_4K, B=3)
+    inp = wl.make_inputs(w, device="cuda")
+    dec = CsaDecoder(inp)
+    dec.build_caches()
+    ref = dec.step().clone()
+    torch.cuda.synchronize()
+    pos = inp.lens.long() - 1
+    bidx = torch.arange(w.B, device="cuda")
+    lay = dec.packed_layout()
+    in_host = torch.zeros(lay["_bytes"], dtype=torch.uint8).pin_memory()
+    for name, src in (("h", inp.h), ("q", inp.q), ("kv_row", inp.raw_kv[bidx, pos]),
+                      ("ki_row", inp.raw_ki[bidx, pos])):
+        off, _, _ = lay[name]
+        flat = src.detach().contiguous().cpu().view(torch.uint8).reshape(-1)
+        assert off % 256 == 0
+        in_host[off:off + flat.numel()] = flat
+    out_host = torch.empty(dec.out.shape, dtype=dec.out.dtype).pin_memory()
+    dec.step_packed(in_host, out_host)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host.view(torch.int16), ref.cpu().view(torch.int16))
+    dec.ws_idx.check()
+    dec.ws_att.check()
