@@ -189,11 +189,12 @@ CSA_API csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
  */
 /*
  * Scoring kernels (csa_index_scores, csa_index_select, csa_index_stage_score,
- * csa_index_topk).  With T >= 256 queries, bf16 keys and Hi in {4, 8, 16}
- * the scores come from a tensor-core (tcgen05) kernel that reads the key
- * cache in whole 128-row tiles: each sequence's cache must then hold
- * max_blocks rows (rows past a query's V are read and ignored; q_seq values
- * must be below CSA_MAX_T).  Fewer queries use the streaming decode kernel,
+ * csa_index_topk).  With T >= 256 queries, bf16 keys, Hi in {4, 8, 16} and
+ * max_blocks >= 128 the scores come from a tensor-core (tcgen05) kernel
+ * that reads the key cache in whole 128-row tiles: each sequence's cache
+ * must then hold max_blocks rows (rows past a query's V are read and
+ * ignored; q_seq values must be below CSA_MAX_T).  Other calls use the
+ * streaming decode kernel,
  * which reads only visible rows.  The two kernels group the products
  * differently, so a query's scores may differ in the last bits between a
  * call below and a call at or above T = 256 (both within the stated score

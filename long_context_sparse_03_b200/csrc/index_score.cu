@@ -842,7 +842,8 @@ __global__ void __launch_bounds__(NTH) rank_kernel(const uint64_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------- host
-bool index_score_umma_applies(int T, int Hi, int fmt, const float* q, const void* kidx, int64_t kstride_bytes);
+bool index_score_umma_applies(int T, int Hi, int fmt, const float* q, const void* kidx, int64_t kstride_bytes,
+                              int max_blocks);
 cudaError_t launch_index_score_umma(const float* q, const float* w, const int* q_seq, const int* q_pos, int T, int Hi,
                                     const void* kidx, int64_t kstride_bytes, int m, int max_blocks, int k,
                                     float* scores, int64_t ld_scores, unsigned* hist, unsigned* thr, unsigned* done,
@@ -918,7 +919,7 @@ cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq,
         if (e != cudaSuccess) return e;
         *launches += 1;
     }
-    if (index_score_umma_applies(T, Hi, fmt, q, kidx, a.kstride_bytes))
+    if (index_score_umma_applies(T, Hi, fmt, q, kidx, a.kstride_bytes, max_blocks))
         e = launch_index_score_umma(q, w, q_seq, q_pos, T, Hi, kidx, a.kstride_bytes, m, max_blocks, k, scores,
                                     ld_scores, hist, thr, done, status, stream);
     else if (fmt == 0) e = nt == 1 ? launch_score_t<0, 1>(a, stream) : launch_score_t<0, 2>(a, stream);

@@ -490,8 +490,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Whether the tensor-core path takes this call (else the decode kernel does).
-bool index_score_umma_applies(int T, int Hi, int fmt, const float* q, const void* kidx, int64_t kstride_bytes) {
-    return fmt == 0 && (Hi == 4 || Hi == 8 || Hi == 16) && T >= 256 && (reinterpret_cast<uintptr_t>(kidx) & 15) == 0 &&
+bool index_score_umma_applies(int T, int Hi, int fmt, const float* q, const void* kidx, int64_t kstride_bytes,
+                              int max_blocks) {
+    return fmt == 0 && (Hi == 4 || Hi == 8 || Hi == 16) && T >= 256 && max_blocks >= kUmTile &&
+           (reinterpret_cast<uintptr_t>(kidx) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(q) & 15) == 0 &&
            kstride_bytes % 16 == 0 && kstride_bytes > 0 && tensor_map_encoder() != nullptr;
 }

@@ -186,7 +186,7 @@ def test_index_scores(oracle, fmt, Hi, N, T):
     (0, 4, 1024, 1, 64, False, False), (0, 8, 3000, 4, 2048, False, False), (0, 8, 2500, 5, 1, False, False),
     (0, 8, 4000, 4, 100, True, False), (0, 8, 4000, 4, 300, False, True), (1, 16, 20000, 2, 1024, False, False),
     (0, 8, 3000, 300, 256, False, False), (0, 8, 4000, 260, 100, True, False), (0, 16, 2500, 300, 512, False, True),
-    (0, 8, 9000, 300, 512, False, False), (0, 4, 9000, 270, 64, True, False)])
+    (0, 8, 9000, 300, 512, False, False), (0, 4, 9000, 270, 64, True, False), (0, 8, 100, 300, 32, False, False)])
 def test_index_select(oracle, fmt, Hi, N, T, k, ties, neg):
     rng = np.random.default_rng(1000 + fmt + Hi + N + k)
     m = 4
