@@ -194,11 +194,11 @@ CSA_API csa_status csa_index_query(const void* h, int T, int D, int r, int Hi,
  * that reads the key cache in whole 128-row tiles: each sequence's cache
  * must then hold max_blocks rows (rows past a query's V are read and
  * ignored; q_seq values must be below CSA_MAX_T).  Other calls use the
- * streaming decode kernel,
- * which reads only visible rows.  The two kernels group the products
- * differently, so a query's scores may differ in the last bits between a
- * call below and a call at or above T = 256 (both within the stated score
- * tolerance); within either regime results do not depend on the batch.
+ * streaming decode kernel, which reads only visible rows.  The two kernels
+ * group the products differently, so a query's scores may differ in the
+ * last bits between a call below and a call at or above T = 256 (both
+ * within the stated score tolerance); within either regime results do not
+ * depend on the batch.
  */
 CSA_API csa_status csa_index_scores(const float* q, const float* w, const int32_t* q_seq,
                             const int32_t* q_pos, int T, int Hi,
