@@ -270,7 +270,7 @@ CSA_API size_t hca_attend_workspace_size(int T, int H, int max_rows);
  * lse fp32 [T][H] (natural log of the softmax denominator, -inf for an
  * empty set) or NULL.  An empty attended set gives out = 0.
  * fp32 logits, softmax and accumulation; split-K over fixed 64-row splits
- * (256-row for hca_attend) merged in a fixed order.
+ * (512-row for hca_attend) merged in a fixed order.
  */
 CSA_API csa_status csa_sparse_attend(const void* q, const int32_t* q_seq, const int32_t* q_pos,
                              int T, int H, const void* comp, int64_t comp_seq_stride,

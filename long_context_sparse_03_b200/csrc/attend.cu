@@ -12,7 +12,7 @@
 // 64-row blocks gathered into shared memory with cp.async (the next block is
 // in flight while this one computes), an online softmax in registers, then
 // O += P V with P re-packed from the S accumulators.  The attended row list
-// of a query is cut into fixed splits (64 rows for CSA, 256 for HCA; never a
+// of a query is cut into fixed splits (64 rows for CSA, 512 for HCA; never a
 // function of the batch).  Each split yields (max, sum, unnormalised output)
 // from a fresh online softmax, and the splits are folded in split order with
 // one fixed formula (fold_split).  Two launch shapes compute exactly the same
@@ -26,7 +26,7 @@
 namespace csa {
 
 constexpr int kCsaRowsPerSplit = 64;    // CSA: k + W rows per query, latency-bound
-constexpr int kHcaRowsPerSplit = 256;   // HCA: thousands of rows per query
+constexpr int kHcaRowsPerSplit = 512;   // HCA: thousands of rows per query
 constexpr int kRowBlock = 64;
 constexpr int kRowStride = 136;  // bf16 per smem row (272 B: conflict-free ldmatrix)
 
