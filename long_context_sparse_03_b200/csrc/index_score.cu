@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(256) zero_state_kernel(unsigned* __restrict__ 
 __device__ __forceinline__ int owner_cta(int64_t x, int64_t U, int64_t G) { return (int)(((x + 1) * G - 1) / U); }
 
 // Persistent, warp-specialised scoring kernel.  CTA c takes work units
-// [u_lo, u_hi) of the flattened (query, 128-key unit) space.  Warp 8 is the
+// [u_lo, u_hi) of the flattened (query, 256-key unit) space.  Warp 8 is the
 // producer: one lane streams each unit's key rows into a ring of shared
 // memory stages with 1-D TMA bulk copies (completion counted on a "full"
 // mbarrier per stage).  Warps 0-7 consume: each scores two 16-key tiles of
