@@ -889,6 +889,7 @@ cudaError_t launch_index_score(const float* q, const float* w, const int* q_seq,
                                int m, int max_blocks, int k, float* scores, int64_t ld_scores, unsigned* hist,
                                unsigned* cnt, unsigned* done, unsigned* thr, unsigned* status, cudaStream_t stream,
                                int* launches) {
+    (void)cnt;   // cleared with the histograms: hist, cnt and done are one contiguous region
     ScoreArgs a;
     a.q = q;
     a.w = w;

@@ -98,7 +98,7 @@ uint8_t oracle_float_to_e4m3_satfinite(float v) {
 #endif
     } else {
         int e;
-        double f = frexp(a, &e);   /* a = f * 2^e */
+        (void)frexp(a, &e);            /* a = f * 2^e with f in [0.5, 1) */
         double q = ldexp(1.0, e - 4);  /* 4 significant bits */
 #if ORACLE_PLANT == 9
         r = floor(a / q) * q;
