@@ -323,8 +323,13 @@ def main():
         tf_peak, tf_src = measured_tensor_peak()
         ach = fl["indexer"] / (k_ms / 1e3) / 1e12
         kname = "zero_state_kernel+index_score_umma_kernel"   # the stage timed by the events
+        # DRAM bytes read + written by the scoring kernel, from an ncu capture of
+        # 2048 of the chunk's queries (profiles/index_score_umma_kernel_prefill_t2048.md:
+        # 25.8 MB read + 232.2 MB written, mostly the fp32 score matrix); the
+        # traffic grows with the queries scored, so x4 for the 8192-query chunk.
+        traffic = 4 * 258_021_888 if args.workload == "csa_prefill_8k" else None
         roof = {"bound": "tensor", "kernel": kname, "achieved": round(ach, 2), "peak": tf_peak,
-                "unit": "TFLOP/s", "frac": round(ach / tf_peak, 4), "peak_source": tf_src, "traffic": None,
+                "unit": "TFLOP/s", "frac": round(ach / tf_peak, 4), "peak_source": tf_src, "traffic": traffic,
                 "algorithmic_flops_per_launch": fl["indexer"], "avg_launch_ms": round(k_ms, 5),
                 "step_flops": fl}
     else:
