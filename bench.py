@@ -211,12 +211,17 @@ def main():
     args.warmup = max(3, args.warmup)
 
     rank, world, local = dist_env()
-    if world > 1:
+    # the reference arm is the CPU oracle: without a GPU it runs on the host alone
+    host_only = args.impl == "reference" and not torch.cuda.is_available()
+    if world > 1 and not host_only:
         import torch.distributed as dist
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+    if host_only:
+        dev = torch.device("cpu")
+    else:
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
 
     w0 = WORKLOADS[args.workload]
     w = wl.scaled(w0, seed=rank_seed(w0.seed, rank))
